@@ -182,6 +182,48 @@ def expert_ffn(rows: np.ndarray, w1: np.ndarray, w2: np.ndarray) -> np.ndarray:
     return h @ np.asarray(w2, dtype=np.float64).T
 
 
+def grouped_ffn(x, perm, offsets, K, w1, w2, ws1=None, ws2=None):
+    """Each expert applied to its dispatched segment, plus the shared expert.
+
+    [MOE-ARCH] §3.1: the dispatcher calls expert[e] on the rows gathered into
+    its part of the shared buffer. Row ``r`` of expert e's segment
+    (offsets[e] <= r < offsets[e+1]) holds copy ``perm[r]`` of token
+    ``perm[r] // K``. The shared expert ([K3-A2A] opening section, resident
+    expert every token passes through) is applied to every token row.
+    Returns (y_rows [T*K, H], y_shared [T, H] or None), float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    perm = np.asarray(perm, dtype=np.int64)
+    H = x.shape[1]
+    y_rows = np.zeros((perm.size, H), dtype=np.float64)
+    for e in range(len(offsets) - 1):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if b > a:
+            y_rows[a:b] = expert_ffn(x[perm[a:b] // K], w1[e], w2[e])
+    y_shared = expert_ffn(x, ws1, ws2) if ws1 is not None else None
+    return y_rows, y_shared
+
+
+def combine(y_rows, w, inv, y_shared=None):
+    """``y[t] = sum_{k<K} w[t,k] * y_rows[inv[t*K+k]] (+ y_shared[t])``.
+
+    [K3-A2A] "物理通信拓扑", combine phase: each token's expert outputs are
+    brought back and summed with their routing weights (the residual the
+    page also adds belongs to the surrounding transformer and is left out);
+    [MOE-ARCH] §3.1: results are scattered back to their original positions.
+    """
+    w = np.asarray(w, dtype=np.float64)
+    T, K = w.shape
+    y_rows = np.asarray(y_rows, dtype=np.float64)
+    inv = np.asarray(inv, dtype=np.int64).reshape(T, K)
+    y = np.zeros((T, y_rows.shape[1]), dtype=np.float64)
+    for k in range(K):
+        y += w[:, k:k + 1] * y_rows[inv[:, k]]
+    if y_shared is not None:
+        y += np.asarray(y_shared, dtype=np.float64)
+    return y
+
+
 # --------------------------------------------------------------------------
 # a9  full layer: route, dispatch, experts, weighted combine (+ shared)
 # --------------------------------------------------------------------------
@@ -301,7 +343,7 @@ def load_stats(counts: np.ndarray, T: int, K: int, cf_num: int = 5, cf_den: int 
         "skew_ratio": float(mx) / (float(mn) + 1e-5),
         "gini": gini_exact(c),
         "overflow": overflow,
-        "overflow_rate": float(overflow) / float(T * K),
+        "overflow_rate": float(overflow) / float(T * K) if T * K else 0.0,
         "num_stragglers": int(np.count_nonzero(c > cap)),
         "straggler_mask": (c > cap).astype(np.uint8),
     }

@@ -348,3 +348,32 @@ def test_stats_on_a_routed_batch_are_consistent():
     assert st["overflow"] == sum(max(0, int(c) - cap) for c in counts)
     assert st["num_stragglers"] == int(st["straggler_mask"].sum())
     assert 0.0 <= st["gini"] < 1.0
+
+
+# ------------------------------------------------ stage-wise formulation ---
+def test_stagewise_grouped_ffn_and_combine_equal_layer_definition():
+    """Dispatch -> per-expert FFN on each segment -> combine gives the same y
+    as the per-token definition, including idle experts and the shared one."""
+    rng = _rng(41)
+    T, H, E, D, K = 23, 16, 9, 20, 3
+    x, wr, w1, w2, ws1, ws2 = _rand_layer(rng, T, H, E, D, Ds=12)
+    bias = -0.8 * np.log(np.arange(E) + 1.0)
+    out = oracle.moe_layer_forward(x, wr, bias, w1, w2, ws1, ws2, K)
+    y_rows, y_sh = oracle.grouped_ffn(x, out["perm"], out["offsets"], K, w1, w2, ws1, ws2)
+    for r in range(T * K):                       # row r is copy perm[r] of token perm[r] // K
+        e = np.searchsorted(out["offsets"], r, side="right") - 1
+        np.testing.assert_allclose(y_rows[r], _torch_ffn(x[out["perm"][r] // K][None], w1[e], w2[e])[0],
+                                   rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(oracle.combine(y_rows, out["w"], out["inv"], y_sh), out["y"],
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_combine_K1_unit_weight_is_inverse_permutation():
+    rng = _rng(42)
+    TK, H = 19, 5
+    rows = rng.normal(size=(TK, H))
+    perm = rng.permutation(TK)
+    inv = np.empty(TK, dtype=np.int64)
+    inv[perm] = np.arange(TK)
+    y = oracle.combine(rows, np.ones((TK, 1)), inv)
+    np.testing.assert_array_equal(y, rows[inv])
