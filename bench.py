@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""MoE layer forward benchmark on B200: tokens/s and fraction of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload c2] [--T 4096] [--no-sweep] [--no-cpu-baseline]
+
+A step is one pass of the whole layer (router + selection, dispatch, grouped
+expert FFN with the shared expert, combine) over one batch of T tokens of the
+chosen workload (default: the Mixtral-shaped bf16 layer, H=4096, E=8, K=2,
+D=14336, at T=4096). Inputs are seeded synthetic tensors resident in HBM
+(1.9 GB of expert weights per step, larger than the 126 MB L2). Under
+torchrun every rank runs an independent replica on its own token batch
+(weak scaling, no data-path collective); timing is the max over ranks.
+
+Rank 0 prints one JSON line. `--impl reference` times the fp64 CPU oracle on
+a bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE layer tokens/s at 1 B200 + % of roofline (HBM GB/s decode, TFLOPS prefill)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default="c2")
+    p.add_argument("--T", type=int, default=None)
+    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--sweep-all", action="store_true", help="also measure every other workload point")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------- workload ---
+def algorithmic(wl, T, touched, counts=None):
+    """Algorithmic FLOPs and HBM bytes of one layer forward (and of the expert
+    GEMMs alone). FLOPs: router 2*T*H*E, routed experts 4*T*K*H*D (2*H*D
+    multiply-adds per copy, from the Kimi K3 page's Time_comp), shared expert
+    4*T*H*Ds. Bytes: router weights, the weights of every expert the routing
+    touched, the shared expert's weights, x in and y out."""
+    es = 2 if wl.dtype == "bf16" else 4
+    H, E, K, D, Ds = wl.H, wl.E, wl.K, wl.D, wl.Ds
+    f_router = 2 * T * H * E
+    f_gemm = 4 * T * K * H * D + 4 * T * H * Ds
+    b_weights = touched * 2 * H * D * es + 2 * H * Ds * es
+    b_layer = E * H * es + b_weights + 2 * T * H * es
+    b_gemm = b_weights + T * H * es * (1 + (1 if Ds else 0)) + T * K * H * es
+    return {"flops": f_router + f_gemm, "bytes": b_layer, "gemm_flops": f_gemm, "gemm_bytes": b_gemm}
+
+
+def roofline_bound(flops, nbytes, peaks):
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    return ("tensor", t_tc) if t_tc >= t_hbm else ("hbm", t_hbm)
+
+
+# --------------------------------------------------------------- clocks ---
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu), "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for r in csv.reader(f):
+                if len(r) >= 9:
+                    rows.append([c.strip() for c in r])
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def build_and_import():
+    """Builds libmoe.so if stale (by file path, before the package loads it)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_moe_build", os.path.join(ROOT, "fine_grained_moe_router_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import fine_grained_moe_router_b200 as M
+    return M
+
+
+# ------------------------------------------------------------ distributed ---
+def dist_info():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------- CPU oracle ---
+def oracle_inputs(wl, host, x):
+    """fp64 widening of the inputs for the oracle (outside any timed region)."""
+    return dict(x=mi.to_f64(x), wr=mi.to_f64(host["w_router"]), bias=host["bias"].numpy(),
+                w1=mi.LazyF64(host["w1"]), w2=mi.LazyF64(host["w2"]),
+                ws1=mi.to_f64(host["ws1"]), ws2=mi.to_f64(host["ws2"]))
+
+
+def widen_all(inp):
+    """Replace lazily widened expert weights by float64 arrays when memory allows."""
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = 0
+    n = len(inp["w1"])
+    need = 2 * n * inp["w1"].t[0].numel() * 8
+    if avail > 3 * need:
+        inp = dict(inp)
+        inp["w1"] = [inp["w1"][e] for e in range(n)]
+        inp["w2"] = [inp["w2"][e] for e in range(n)]
+    return inp
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(wl, inp, T, n_tokens, seed):
+    import oracle
+    tokens = mi.sample_tokens(T, n_tokens, seed).numpy()
+    t0 = time.perf_counter()
+    oracle.moe_layer_forward(inp["x"], inp["wr"], inp["bias"], inp["w1"], inp["w2"], inp["ws1"],
+                             inp["ws2"], wl.K, tokens=tokens)
+    return time.perf_counter() - t0, len(tokens)
+
+
+def default_sample(wl, T):
+    # about 10-30 s of fp64 work on the host for the cpu_baseline leg
+    return min(T, 256 if wl.E <= 16 else 128)
+
+
+# ------------------------------------------------------------ reference ---
+def run_reference(args, wl, T):
+    rank, world, _ = dist_info()
+    if rank != 0:
+        return
+    host = mi.draw_layer(wl)
+    x = mi.draw_x(wl, T)
+    inp = widen_all(oracle_inputs(wl, host, x))
+    n = min(T, 16)
+    for i in range(args.warmup):
+        time_oracle(wl, inp, T, n, seed=100 + i)
+    times = []
+    for i in range(args.steps):
+        dt, n_done = time_oracle(wl, inp, T, n, seed=200 + i)
+        times.append(dt)
+    total = sum(times)
+    value = n * args.steps / total
+    sample = (f"per step: routing of all {T} tokens + expert FFNs of {n} seeded sample tokens "
+              f"(fp64 numpy oracle)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, T, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, T, world):
+    return {"workload": f"{wl.name}: H={wl.H} E={wl.E} K={wl.K} D={wl.D} Ds={wl.Ds} T={T} ({wl.key})",
+            "T": T, "H": wl.H, "E": wl.E, "K": wl.K, "D": wl.D, "Ds": wl.Ds,
+            "global_batch": T * world, "l2": "inputs larger than L2 (expert weights "
+            f"{2 * wl.E * wl.H * wl.D * (2 if wl.dtype == 'bf16' else 4) / 1e9:.2f} GB per step)",
+            "parallelism": f"replicas x{world} (independent token batches, no collective)"}
+
+
+# ----------------------------------------------------------------- ours ---
+class Runner:
+    def __init__(self, M, wl, dev, T, replica):
+        self.M, self.wl, self.T = M, wl, T
+        self.desc = M.make_desc(T, wl.H, wl.E, wl.K, wl.D, wl.Ds,
+                                M.MOE_BF16 if wl.dtype == "bf16" else M.MOE_F32)
+        self.dev = dev
+        self.weights = M.make_weights(dev["w_router"], dev["w1"], dev["w2"], dev["ws1"], dev["ws2"],
+                                      dev["bias"])
+        self.ws = M.alloc_workspace(self.desc)
+        self.x_host = mi.draw_x(wl, T, replica)
+        self.x = self.x_host.cuda()
+        self.y = torch.empty_like(self.x)
+        self.counts = torch.empty(wl.E, dtype=torch.int32, device="cuda")
+        self.routing = M.make_routing(counts=self.counts)
+
+    def step(self):
+        self.M.moe_layer_forward(self.desc, self.weights, self.x, self.y, self.routing, self.ws)
+
+    def timed(self, steps, warmup, world, device, stage_events=False):
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        n0 = self.M.moe_kernel_launch_count()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(steps):
+            self.step()
+        end.record()
+        torch.cuda.synchronize()
+        launches = self.M.moe_kernel_launch_count() - n0
+        barrier(world)
+        ms = max_over_ranks(start.elapsed_time(end), world, device)
+        return ms, launches
+
+    def stages(self, steps):
+        """Per-stage device times (ms, mean over steps) from events recorded
+        between the kernels of moe_layer_forward_profiled."""
+        M = self.M
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        for s in range(steps):
+            M.moe_layer_forward_profiled(self.desc, self.weights, self.x, self.y, self.routing, self.ws, evs[s])
+        torch.cuda.synchronize()
+        out = {}
+        for i, name in enumerate(M.FORWARD_STAGES):
+            out[name] = statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(steps))
+        return out
+
+    def e2e(self, steps, warmup, world, device):
+        """Through the public API from pinned host memory: H2D of x, forward,
+        D2H of y, every step."""
+        xh = self.x_host.pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+
+        def one():
+            self.x.copy_(xh, non_blocking=True)
+            self.step()
+            yh.copy_(self.y, non_blocking=True)
+
+        for _ in range(warmup):
+            one()
+        torch.cuda.synchronize()
+        barrier(world)
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(steps):
+            one()
+        end.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = max_over_ranks(start.elapsed_time(end), world, device)
+        nbytes = xh.numel() * xh.element_size()
+        return ms, nbytes, yh.numel() * yh.element_size()
+
+    def touched(self):
+        return int((self.counts > 0).sum().item())
+
+
+def run_ours(args, wl, T):
+    rank, world, local = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    M = build_and_import()
+    peaks, peaks_src = load_peaks()
+
+    host = mi.draw_layer(wl)
+    dev = {k: (v.to(device) if v is not None else None) for k, v in host.items()}
+    R = Runner(M, wl, dev, T, replica=rank)
+
+    sampler = ClockSampler(device.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    sampler.start()
+    ms, launches = R.timed(args.steps, args.warmup, world, device)
+    clocks = sampler.stop()
+    ms_step = ms / args.steps
+    value = world * T * args.steps / (ms / 1e3)
+
+    stages = R.stages(args.steps)
+    touched = R.touched()
+    alg = algorithmic(wl, T, touched)
+    gemm_ms = stages["gemm1"] + stages["gemm2"]
+    bound, _ = roofline_bound(alg["gemm_flops"], alg["gemm_bytes"], peaks)
+    if bound == "tensor":
+        achieved = alg["gemm_flops"] / (gemm_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    else:
+        achieved = alg["gemm_bytes"] / (gemm_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    lbound, t_roof = roofline_bound(alg["flops"], alg["bytes"], peaks)
+
+    e2e_ms, h2d, d2h = R.e2e(args.steps, args.warmup, world, device)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded: x ~ N(0,1), weights ~ N(0,1/fan_in) in bf16, Zipf logit skew "
+                "as a bias input where the workload has one)",
+        "config": workload_config(wl, T, world),
+        "roofline": {"kernel": "grouped expert GEMMs (GEMM1 + GeLU, GEMM2; shared expert included)",
+                     "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": None, "peak_source": peaks_src,
+                     "ms_per_launch_pair": gemm_ms},
+        "layer_roofline": {"bound": lbound, "t_roof_ms": 1e3 * t_roof, "frac": 1e3 * t_roof / ms_step,
+                           "flops": alg["flops"], "bytes": alg["bytes"], "experts_touched": touched},
+        "stages_ms": stages,
+        "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if not args.no_sweep and world == 1:
+        line["sweep"] = sweep(M, wl, dev, T, peaks, args.sweep_all)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, host, R.x_host, T)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def measure_point(M, wl, dev, T, peaks, steps=20, warmup=5):
+    R = Runner(M, wl, dev, T, replica=0)
+    ms, _ = R.timed(steps, warmup, 1, None)
+    st = R.stages(steps)
+    alg = algorithmic(wl, T, R.touched())
+    bound, t_roof = roofline_bound(alg["flops"], alg["bytes"], peaks)
+    ms_step = ms / steps
+    return {"workload": wl.key, "T": T, "tokens_per_s": T / (ms_step / 1e3), "us_per_step": 1e3 * ms_step,
+            "bound": bound, "roofline_us": 1e6 * t_roof, "frac": 1e3 * t_roof / ms_step,
+            "experts_touched": R.touched(), "stages_us": {k: 1e3 * v for k, v in st.items()}}
+
+
+def sweep(M, wl, dev, T_main, peaks, all_workloads):
+    out = [measure_point(M, wl, dev, T, peaks) for T in wl.Ts if T != T_main]
+    if all_workloads:
+        for key in ("c3", "c4", "c5", "c1"):
+            if key == wl.key:
+                continue
+            w2 = mi.WORKLOADS[key]
+            host = mi.draw_layer(w2)
+            d2 = {k: (v.cuda() if v is not None else None) for k, v in host.items()}
+            for T in w2.Ts:
+                out.append(measure_point(M, w2, d2, T, peaks))
+            del d2
+            torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline(wl, host, x, T):
+    inp = widen_all(oracle_inputs(wl, host, x))
+    n = default_sample(wl, T)
+    dt, n_done = time_oracle(wl, inp, T, n, seed=7)
+    return {"value": n_done / dt, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"routing of all {T} tokens + expert FFNs of {n_done} seeded sample tokens "
+                      f"(fp64 numpy oracle, {dt:.1f} s)"}
+
+
+def main():
+    args = parse_args()
+    wl = mi.WORKLOADS[args.workload]
+    T = args.T if args.T is not None else max(wl.Ts)
+    if args.impl == "reference":
+        run_reference(args, wl, T)
+    else:
+        run_ours(args, wl, T)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,328 @@
+// C ABI of libmoe: argument checks, workspace layout and the launch sequence.
+// Every compute step runs in this library's kernels; nothing here computes
+// on the host except sizes.
+#include <atomic>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+size_t dtype_size(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
+
+static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+WsLayout workspace_layout(const moe_layer_desc& d) {
+  WsLayout L{};
+  const size_t T = d.T, K = d.K, E = d.E, H = d.H, D = d.D, Ds = d.Ds;
+  const size_t TK = T * K;
+  const size_t es = dtype_size(d.dtype);
+  L.n_chunks = (int)std::max<size_t>(1, (TK + kChunk - 1) / kChunk);
+  const size_t rows_bound = std::min(E, TK);          // groups that can hold rows
+  L.max_tiles_simt = (int)((TK + kSimtRows - 1) / kSimtRows + rows_bound +
+                           (Ds ? (T + kSimtRows - 1) / kSimtRows : 0));
+  const size_t rt_routed = (TK + kTcRows - 1) / kTcRows + rows_bound;
+  const size_t rt_shared = Ds ? (T + kTcRows - 1) / kTcRows : 0;
+  L.max_tiles_tc1 = (int)(rt_routed * (D / 128) + rt_shared * (Ds / 128));
+  L.max_tiles_tc2 = (int)((rt_routed + rt_shared) * (H / 128));
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.hdr = take(sizeof(WsHeader));
+  L.hist = take(sizeof(int32_t) * L.n_chunks * E);
+  L.base = take(sizeof(int32_t) * L.n_chunks * E);
+  L.tiles_simt = take(sizeof(Tile) * std::max(1, L.max_tiles_simt));
+  L.tiles_tc1 = take(sizeof(Tile) * std::max(1, L.max_tiles_tc1));
+  L.tiles_tc2 = take(sizeof(Tile) * std::max(1, L.max_tiles_tc2));
+  L.idx = take(sizeof(int32_t) * TK);
+  L.w = take(sizeof(float) * TK);
+  L.counts = take(sizeof(int32_t) * E);
+  L.offsets = take(sizeof(int32_t) * (E + 1));
+  L.perm = take(sizeof(int32_t) * TK);
+  L.inv = take(sizeof(int32_t) * TK);
+  L.logits = take(sizeof(float) * T * E);
+  L.xp = take(d.dtype == MOE_BF16 ? es * TK * H : 0);
+  L.hm = take(es * TK * D);
+  L.hs = take(es * T * Ds);
+  L.yr = take(es * TK * H);
+  L.ys = take(es * T * H * (Ds ? 1 : 0));
+  L.stats = take(sizeof(moe_stats) + E);
+  L.total = o;
+  return L;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static moe_status check_desc(const moe_layer_desc* d) {
+  if (!d) return MOE_ERR_INVALID_ARG;
+  if (d->T < 0 || d->H < 1 || d->E < 1 || d->K < 1 || d->D < 1 || d->Ds < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (d->dtype != MOE_F32 && d->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (d->cf_num < 0 || d->cf_den < 1) return MOE_ERR_INVALID_ARG;
+  if (d->K > d->E) return MOE_ERR_INVALID_ARG;
+  if (d->K > kMaxK || d->E > kMaxE) return MOE_ERR_UNSUPPORTED;
+  const int q = (d->dtype == MOE_BF16) ? 128 : 4;
+  if (d->H % q || d->D % q || d->Ds % q) return MOE_ERR_UNSUPPORTED;
+  if ((long long)d->T * d->K > (1LL << 30)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+static moe_status check_ws(const moe_layer_desc& d, const void* ws, size_t ws_bytes) {
+  if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < workspace_layout(d).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+// All listed pointers must be non-null and 16-byte aligned.
+static moe_status check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+static int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = v > 0 ? v : 148;
+  }
+  return cached[dev];
+}
+
+#define MOE_TRY(expr)                 \
+  do {                                \
+    moe_status _s = (expr);           \
+    if (_s != MOE_OK) return _s;      \
+  } while (0)
+
+// Grouped FFN body shared by moe_grouped_ffn and moe_layer_forward. The
+// tile lists must already be in the workspace.
+static moe_status run_grouped_ffn(const moe_layer_desc& d, const WsLayout& L, char* ws,
+                                  const void* x, const int32_t* perm, const void* w1,
+                                  const void* w2, const void* ws1, const void* ws2, void* y_rows,
+                                  void* y_shared, cudaStream_t st,
+                                  cudaEvent_t const* ev_after_gemm1 = nullptr) {
+  if (d.T == 0) return MOE_OK;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
+  void* hm = ws + L.hm;
+  void* hs = ws + L.hs;
+  const bool shared = d.Ds > 0;
+  SimtProblem r1{x, perm, d.K, w1, (size_t)d.D * d.H, hm, d.H, d.D};
+  SimtProblem s1{x, nullptr, 1, ws1, 0, hs, d.H, d.Ds};
+  SimtProblem r2{hm, nullptr, 1, w2, (size_t)d.H * d.D, y_rows, d.D, d.H};
+  SimtProblem s2{hs, nullptr, 1, ws2, 0, y_shared, d.Ds, d.H};
+  const Tile* tiles = reinterpret_cast<const Tile*>(ws + L.tiles_simt);
+  MOE_CUDA_TRY(launch_grouped_gemm_simt(d.dtype, true, r1, s1, d.E, tiles, &hdr->n_tiles[0],
+                                        L.max_tiles_simt, std::max(d.D, shared ? d.Ds : 0), st));
+  if (ev_after_gemm1) MOE_CUDA_TRY(cudaEventRecord(*ev_after_gemm1, st));
+  MOE_CUDA_TRY(launch_grouped_gemm_simt(d.dtype, false, r2, s2, d.E, tiles, &hdr->n_tiles[0],
+                                        L.max_tiles_simt, d.H, st));
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_layer_desc* desc) {
+  if (check_desc(desc) != MOE_OK) return 0;
+  return workspace_layout(*desc).total;
+}
+
+moe_status moe_router_topk(const moe_layer_desc* desc, const void* x, const void* w_router,
+                           const float* bias, float* logits_or_null, int32_t* topk_idx,
+                           float* topk_w, void* ws, size_t ws_bytes, moe_stream stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc& d = *desc;
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  if (d.T == 0) return MOE_OK;
+  MOE_TRY(check_ptrs({x, w_router, topk_idx, topk_w}));
+  if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  if (logits_or_null && !aligned16(logits_or_null)) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = workspace_layout(d);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* logits = logits_or_null ? logits_or_null
+                                 : reinterpret_cast<float*>(static_cast<char*>(ws) + L.logits);
+  MOE_CUDA_TRY(launch_gate_logits(d, x, w_router, logits, st));
+  MOE_CUDA_TRY(launch_topk_select(d, logits, bias, topk_idx, topk_w, st));
+  return MOE_OK;
+}
+
+moe_status moe_topk_from_logits(const moe_layer_desc* desc, const float* logits,
+                                const float* bias, int32_t* topk_idx, float* topk_w,
+                                moe_stream stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc& d = *desc;
+  if (d.T == 0) return MOE_OK;
+  MOE_TRY(check_ptrs({logits, topk_idx, topk_w}));
+  if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(launch_topk_select(d, logits, bias, topk_idx, topk_w,
+                                  static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_dispatch(const moe_layer_desc* desc, const int32_t* topk_idx, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
+                        size_t ws_bytes, moe_stream stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc& d = *desc;
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  MOE_TRY(check_ptrs({counts, offsets}));
+  if (d.T > 0) MOE_TRY(check_ptrs({topk_idx, perm, inv}));
+  const WsLayout L = workspace_layout(d);
+  MOE_CUDA_TRY(launch_dispatch(d, L, static_cast<char*>(ws), topk_idx, counts, offsets, perm,
+                               inv, false, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_grouped_ffn(const moe_layer_desc* desc, const void* x, const int32_t* perm,
+                           const int32_t* offsets, const void* w1, const void* w2,
+                           const void* ws1, const void* ws2, void* y_rows, void* y_shared,
+                           void* ws, size_t ws_bytes, moe_stream stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc& d = *desc;
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  if (d.T == 0) return MOE_OK;
+  MOE_TRY(check_ptrs({x, perm, offsets, w1, w2, y_rows}));
+  if (d.Ds > 0) MOE_TRY(check_ptrs({ws1, ws2, y_shared}));
+  const WsLayout L = workspace_layout(d);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  MOE_CUDA_TRY(launch_tiles_from_offsets(d, L, w, offsets, false, st));
+  return run_grouped_ffn(d, L, w, x, perm, w1, w2, ws1, ws2, y_rows, y_shared, st);
+}
+
+moe_status moe_combine(const moe_layer_desc* desc, const void* y_rows, const float* topk_w,
+                       const int32_t* inv, const void* y_shared_or_null, void* y,
+                       moe_stream stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc& d = *desc;
+  if (d.T == 0) return MOE_OK;
+  MOE_TRY(check_ptrs({y_rows, topk_w, inv, y}));
+  if (y_shared_or_null && !aligned16(y_shared_or_null)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(launch_combine(d, y_rows, topk_w, inv, y_shared_or_null, y,
+                              static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer_weights* weights,
+                                     const void* x, void* y, const moe_routing* routing_or_null,
+                                     void* ws, size_t ws_bytes, cudaStream_t st,
+                                     cudaEvent_t const* ev, int n_ev) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc& d = *desc;
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  if (!weights) return MOE_ERR_INVALID_ARG;
+  if (ev && n_ev < kForwardEvents) return MOE_ERR_INVALID_ARG;
+  if (d.T == 0) return MOE_OK;
+  const moe_layer_weights& W = *weights;
+  MOE_TRY(check_ptrs({x, y, W.w_router, W.w1, W.w2}));
+  if (d.Ds > 0) MOE_TRY(check_ptrs({W.ws1, W.ws2}));
+  if (W.expert_bias && !aligned16(W.expert_bias)) return MOE_ERR_INVALID_ARG;
+  moe_routing R{};
+  if (routing_or_null) R = *routing_or_null;
+  for (const void* p : {(const void*)R.topk_idx, (const void*)R.topk_w, (const void*)R.counts,
+                        (const void*)R.offsets, (const void*)R.perm, (const void*)R.inv,
+                        (const void*)R.logits})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = workspace_layout(d);
+  char* w = static_cast<char*>(ws);
+  float* logits = R.logits ? R.logits : reinterpret_cast<float*>(w + L.logits);
+  int32_t* idx = R.topk_idx ? R.topk_idx : reinterpret_cast<int32_t*>(w + L.idx);
+  float* tw = R.topk_w ? R.topk_w : reinterpret_cast<float*>(w + L.w);
+  int32_t* counts = R.counts ? R.counts : reinterpret_cast<int32_t*>(w + L.counts);
+  int32_t* offsets = R.offsets ? R.offsets : reinterpret_cast<int32_t*>(w + L.offsets);
+  int32_t* perm = R.perm ? R.perm : reinterpret_cast<int32_t*>(w + L.perm);
+  int32_t* inv = R.inv ? R.inv : reinterpret_cast<int32_t*>(w + L.inv);
+  void* yr = w + L.yr;
+  void* ys = d.Ds > 0 ? static_cast<void*>(w + L.ys) : nullptr;
+  auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
+
+  MOE_CUDA_TRY(mark(0));
+  MOE_CUDA_TRY(launch_gate_logits(d, x, W.w_router, logits, st));
+  MOE_CUDA_TRY(launch_topk_select(d, logits, W.expert_bias, idx, tw, st));
+  MOE_CUDA_TRY(mark(1));
+  MOE_CUDA_TRY(launch_dispatch(d, L, w, idx, counts, offsets, perm, inv, false, st));
+  MOE_CUDA_TRY(mark(2));
+  MOE_TRY(run_grouped_ffn(d, L, w, x, perm, W.w1, W.w2, W.ws1, W.ws2, yr, ys, st,
+                          ev ? ev + 3 : nullptr));
+  MOE_CUDA_TRY(mark(4));
+  MOE_CUDA_TRY(launch_combine(d, yr, tw, inv, ys, y, st));
+  MOE_CUDA_TRY(mark(5));
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* weights,
+                             const void* x, void* y, const moe_routing* routing_or_null,
+                             void* ws, size_t ws_bytes, moe_stream stream) {
+  return layer_forward_impl(desc, weights, x, y, routing_or_null, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream), nullptr, 0);
+}
+
+moe_status moe_layer_forward_profiled(const moe_layer_desc* desc,
+                                      const moe_layer_weights* weights, const void* x, void* y,
+                                      const moe_routing* routing_or_null, void* ws,
+                                      size_t ws_bytes, moe_stream stream,
+                                      void* const* stage_events, int n_events) {
+  if (!stage_events) return MOE_ERR_INVALID_ARG;
+  return layer_forward_impl(desc, weights, x, y, routing_or_null, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream),
+                            reinterpret_cast<cudaEvent_t const*>(stage_events), n_events);
+}
+
+moe_status moe_expert_stats(const moe_layer_desc* desc, const int32_t* counts,
+                            uint8_t* straggler_mask_or_null, moe_stats* out_host, void* ws,
+                            size_t ws_bytes, moe_stream stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc& d = *desc;
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  if (!counts || !out_host) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = workspace_layout(d);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  moe_stats* dev = reinterpret_cast<moe_stats*>(static_cast<char*>(ws) + L.stats);
+  MOE_CUDA_TRY(launch_expert_stats(d, counts, straggler_mask_or_null, dev, st));
+  MOE_CUDA_TRY(cudaMemcpyAsync(out_host, dev, sizeof(moe_stats), cudaMemcpyDeviceToHost, st));
+  MOE_CUDA_TRY(cudaStreamSynchronize(st));
+  return MOE_OK;
+}
+
+moe_status moe_check_status(void* ws, size_t ws_bytes, moe_stream stream) {
+  if (!ws || ws_bytes < sizeof(WsHeader)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t status = 0;
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  MOE_CUDA_TRY(cudaMemcpyAsync(&status, &hdr->status, sizeof(status), cudaMemcpyDeviceToHost, st));
+  MOE_CUDA_TRY(cudaMemsetAsync(&hdr->status, 0, sizeof(uint32_t), st));
+  MOE_CUDA_TRY(cudaStreamSynchronize(st));
+  if (status & kStatusTimeout) return MOE_ERR_TIMEOUT;
+  if (status & kStatusBadIndex) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+uint64_t moe_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA launch or runtime error";
+    case MOE_ERR_TIMEOUT: return "a bounded device wait ran out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

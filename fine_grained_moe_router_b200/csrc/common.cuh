@@ -1,0 +1,77 @@
+// Shared device/host helpers of libmoe (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <climits>
+#include <algorithm>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kMaxK = 16;
+constexpr int kMaxE = 512;
+constexpr int kForwardEvents = 6;   // stage events of moe_layer_forward_profiled
+
+// Status bits written by kernels into the workspace header.
+constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusBadIndex = 2u;   // a top-K index outside [0, E)
+
+// Element access for the two layer dtypes.
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// Exact GeLU 0.5 z (1 + erf(z / sqrt 2)) with CUDA's erff.
+__device__ __forceinline__ float gelu_erf(float z) {
+  return 0.5f * z * (1.0f + erff(z * 0.70710678118654752440f));
+}
+
+// Workspace header: control words the kernels share. Lives at offset 0.
+struct WsHeader {
+  uint32_t status;          // kStatus* bits, cleared by moe_check_status
+  int32_t n_tiles[4];       // tile-list lengths written by the scan kernel
+  uint32_t tickets[8];      // self-resetting arrival counters
+  uint32_t pad[51];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+// One unit of grouped-GEMM work: rows [r0, r0 + n) of group g.
+// g < E: routed expert g (rows of the dispatched buffer);
+// g == E: the shared expert (token rows).
+struct Tile {
+  int32_t g;
+  int32_t r0;
+  int32_t n;
+  int32_t m0;   // first output column (weight row) of the tile; used by the tensor-core path
+};
+
+// Offsets of each workspace region (bytes), 256-byte aligned.
+struct WsLayout {
+  size_t hdr, hist, base, tiles_simt, tiles_tc1, tiles_tc2, idx, w, counts, offsets, perm, inv,
+      logits, xp, hm, hs, yr, ys, stats, total;
+  int n_chunks;
+  int max_tiles_simt, max_tiles_tc1, max_tiles_tc2;
+};
+
+constexpr int kChunk = 2048;       // copies per dispatch chunk
+constexpr int kSimtRows = 64;      // rows per SIMT FFN tile
+constexpr int kTcRows = 256;       // max rows (MMA N) per tensor-core tile
+
+WsLayout workspace_layout(const moe_layer_desc& d);
+void count_launch();   // bumps the process-wide kernel launch counter
+size_t dtype_size(int dtype);
+
+}  // namespace moe
+
+#define MOE_CUDA_TRY(expr)                                      \
+  do {                                                          \
+    cudaError_t _e = (expr);                                    \
+    if (_e != cudaSuccess) return MOE_ERR_CUDA;                 \
+  } while (0)

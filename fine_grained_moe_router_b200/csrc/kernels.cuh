@@ -1,0 +1,40 @@
+// Internal launcher declarations shared by the C-ABI translation unit.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// One side (routed experts or shared expert) of a grouped GEMM on CUDA cores.
+struct SimtProblem {
+  const void* A;           // activation rows [*, Kd]
+  const int32_t* perm;     // non-null: row r reads A row perm[r] / k_top
+  int k_top;
+  const void* B;           // weights [groups, N, Kd] (group stride b_group_stride elements)
+  size_t b_group_stride;
+  void* C;                 // output rows [*, N]
+  int Kd;                  // reduction length
+  int N;                   // output columns
+};
+
+cudaError_t launch_gate_logits(const moe_layer_desc& d, const void* x, const void* wr,
+                               float* logits, cudaStream_t st);
+cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, const float* bias,
+                               int32_t* idx, float* w, cudaStream_t st);
+cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws,
+                            const int32_t* idx, int32_t* counts, int32_t* offsets,
+                            int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st);
+cudaError_t launch_tiles_from_offsets(const moe_layer_desc& d, const WsLayout& L, char* ws,
+                                      const int32_t* offsets, bool tc_tiles, cudaStream_t st);
+cudaError_t launch_gather_rows(const moe_layer_desc& d, const void* x, const int32_t* perm,
+                               void* xp, int num_sms, cudaStream_t st);
+cudaError_t launch_grouped_gemm_simt(int dtype, bool gelu, const SimtProblem& routed,
+                                     const SimtProblem& shared, int E, const Tile* tiles,
+                                     const int* n_tiles, int max_tiles, int max_n,
+                                     cudaStream_t st);
+cudaError_t launch_combine(const moe_layer_desc& d, const void* y_rows, const float* w,
+                           const int32_t* inv, const void* y_shared, void* y, cudaStream_t st);
+cudaError_t launch_expert_stats(const moe_layer_desc& d, const int32_t* counts, uint8_t* mask,
+                                moe_stats* out_dev, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,200 @@
+// Router: gate logits and the top-K selection with renormalised weights.
+//
+// Gate: l = x W_r^T, a bias-free Linear(H, E) ("Kimi K3 fine-grained MoE
+// under high concurrency", FineGrainedMoERouter; "MoE architecture in
+// production" §2.3). Selection: scores Softmax(l + B) with the dynamic
+// expert bias B ("Kimi K3 专家路由不均衡诊断" §四), the top K of them, and
+// the K weights divided by their sum (same router code). The decision is
+// taken on the fp32 values s = l + B: softmax is strictly increasing, so the
+// chosen set is the same, and ties stay exact ties (lower expert index wins).
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// Gate logits on CUDA cores: one warp per expert row, 8 experts x 8 tokens
+// per CTA. W_r rows are read once per token block; x rows come from L2.
+// ---------------------------------------------------------------------------
+template <typename TIn>
+struct Vec;
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  using T = float4;
+  __device__ static void unpack(const T& v, float* f) { f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w; }
+};
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  using T = uint4;
+  __device__ static void unpack(const T& v, float* f) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 q = __bfloat1622float2(p[i]);
+      f[2 * i] = q.x;
+      f[2 * i + 1] = q.y;
+    }
+  }
+};
+
+constexpr int kGateTok = 8;   // tokens per CTA
+constexpr int kGateExp = 8;   // experts per CTA (one per warp)
+
+template <typename TIn>
+__global__ void __launch_bounds__(256) gate_logits_simt(const TIn* __restrict__ x,
+                                                        const TIn* __restrict__ wr,
+                                                        float* __restrict__ logits, int T,
+                                                        int H, int E) {
+  using V = Vec<TIn>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * kGateExp + warp;
+  const int t0 = blockIdx.y * kGateTok;
+  if (e >= E) return;
+  float acc[kGateTok];
+#pragma unroll
+  for (int i = 0; i < kGateTok; ++i) acc[i] = 0.f;
+  const TIn* wrow = wr + (size_t)e * H;
+  for (int h = lane * V::N; h < H; h += 32 * V::N) {
+    float wv[V::N], xv[V::N];
+    V::unpack(*reinterpret_cast<const typename V::T*>(wrow + h), wv);
+#pragma unroll
+    for (int i = 0; i < kGateTok; ++i) {
+      const int t = t0 + i;
+      if (t < T) {
+        V::unpack(*reinterpret_cast<const typename V::T*>(x + (size_t)t * H + h), xv);
+#pragma unroll
+        for (int j = 0; j < V::N; ++j) acc[i] = fmaf(xv[j], wv[j], acc[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kGateTok; ++i) {
+    float v = acc[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    acc[i] = v;
+  }
+  if (lane < kGateTok && t0 + lane < T) {
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < kGateTok; ++i)
+      if (i == lane) v = acc[i];
+    logits[(size_t)(t0 + lane) * E + e] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Top-K selection: one warp per token, lane j holds experts j, j+32, ...
+// K rounds of a warp arg-max by shuffles; the order is (score descending,
+// expert index ascending), so ties go to the lower index and -0.0 == +0.0.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool better(float sa, int ea, float sb, int eb) {
+  return sa > sb || (sa == sb && ea < eb);
+}
+
+template <int NJ>
+__device__ __forceinline__ void select_row(const float* __restrict__ lrow,
+                                           const float* __restrict__ bias, int E, int K,
+                                           int32_t* __restrict__ idx_out,
+                                           float* __restrict__ w_out) {
+  const int lane = threadIdx.x & 31;
+  float s[NJ];
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int e = lane + 32 * j;
+    if (e < E) {
+      const float b = bias ? bias[e] : 0.f;
+      s[j] = __fadd_rn(lrow[e], b);
+    } else {
+      s[j] = -INFINITY;
+    }
+  }
+  uint32_t taken = 0;
+  float my_s = -INFINITY;   // score of slot `lane` (lane < K)
+  int my_e = 0;
+  for (int k = 0; k < K; ++k) {
+    float bs = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !((taken >> j) & 1u) && better(s[j], e, bs, be)) {
+        bs = s[j];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (better(os, oe, bs, be)) {
+        bs = os;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == k) {
+      my_s = bs;
+      my_e = be;
+    }
+  }
+  // w_k = exp(s_k - s_0) / sum_{j<K} exp(s_j - s_0), summed in slot order.
+  const float s0 = __shfl_sync(0xffffffffu, my_s, 0);
+  const float z = (lane < K) ? expf(my_s - s0) : 0.f;
+  float den = 0.f;
+  for (int j = 0; j < K; ++j) den += __shfl_sync(0xffffffffu, z, j);
+  if (lane < K) {
+    idx_out[lane] = my_e;
+    w_out[lane] = z / den;
+  }
+}
+
+template <int NJ>
+__global__ void __launch_bounds__(256) topk_select_kernel(const float* __restrict__ logits,
+                                                          const float* __restrict__ bias, int T,
+                                                          int E, int K,
+                                                          int32_t* __restrict__ idx,
+                                                          float* __restrict__ w) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  select_row<NJ>(logits + (size_t)t * E, bias, E, K, idx + (size_t)t * K, w + (size_t)t * K);
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+cudaError_t launch_gate_logits(const moe_layer_desc& d, const void* x, const void* wr,
+                               float* logits, cudaStream_t st) {
+  if (d.T == 0) return cudaSuccess;
+  dim3 grid((d.E + kGateExp - 1) / kGateExp, (d.T + kGateTok - 1) / kGateTok);
+  count_launch();
+  if (d.dtype == MOE_BF16)
+    gate_logits_simt<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)wr, logits, d.T, d.H, d.E);
+  else
+    gate_logits_simt<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)wr, logits,
+                                                  d.T, d.H, d.E);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, const float* bias,
+                               int32_t* idx, float* w, cudaStream_t st) {
+  if (d.T == 0) return cudaSuccess;
+  const int nj = (d.E + 31) / 32;
+  dim3 grid((d.T + 7) / 8);
+#define MOE_TOPK_CASE(NJ) \
+  case NJ: count_launch(); topk_select_kernel<NJ><<<grid, 256, 0, st>>>(logits, bias, d.T, d.E, d.K, idx, w); break;
+  switch (nj) {
+    MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4)
+    MOE_TOPK_CASE(5) MOE_TOPK_CASE(6) MOE_TOPK_CASE(7) MOE_TOPK_CASE(8)
+    MOE_TOPK_CASE(9) MOE_TOPK_CASE(10) MOE_TOPK_CASE(11) MOE_TOPK_CASE(12)
+    MOE_TOPK_CASE(13) MOE_TOPK_CASE(14) MOE_TOPK_CASE(15) MOE_TOPK_CASE(16)
+    default: return cudaErrorInvalidValue;
+  }
+#undef MOE_TOPK_CASE
+  return cudaGetLastError();
+}
+
+}  // namespace moe

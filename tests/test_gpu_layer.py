@@ -1,0 +1,152 @@
+"""Whole-layer parity (moe_layer_forward through the C ABI) on every workload,
+against the fp64 oracle on the same seeded inputs.
+
+Small token counts are compared on every token; the large ones (T = 512 and
+4096 of the Mixtral-shaped layer, T = 16384 of the prefill layer) on a seeded
+sample of tokens the oracle computes one by one, while routing, dispatch and
+statistics are compared over all tokens. Launch configuration and workspace
+are the ones the benchmark uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+from parity import (DeviceLayer, check_dispatch_valid, compare_routing, rel_max_err, stats_equal,
+                    to_np, y_tol)
+
+pytestmark = pytest.mark.gpu
+
+FULL_POINTS = [("c1", 64), ("c2", 1), ("c2", 8), ("c2", 64), ("c3", 1), ("c3", 16), ("c3", 32),
+               ("c3", 64), ("c3", 128), ("c4", 16), ("c4", 64), ("c4", 128), ("c4", 256)]
+SAMPLED_POINTS = [("c2", 512, 64), ("c2", 4096, 64), ("c5", 16384, 128)]
+
+_cache = {}
+
+
+@pytest.fixture(scope="module")
+def M():
+    from _lib import build_and_import
+    return build_and_import()
+
+
+def layer(key):
+    if key not in _cache:
+        _cache.clear()                     # keep one workload's weights resident at a time
+        torch.cuda.empty_cache()
+        _cache[key] = DeviceLayer(mi.WORKLOADS[key])
+    return _cache[key]
+
+
+def run_and_check(M, L, T, sample=None, replica=0):
+    wl = L.wl
+    x = mi.draw_x(wl, T, replica)
+    xd = x.cuda()
+    d = L.desc(M, T)
+    ws = M.alloc_workspace(d)
+    E, K = wl.E, wl.K
+    r = {
+        "topk_idx": torch.empty((T, K), dtype=torch.int32, device="cuda"),
+        "topk_w": torch.empty((T, K), dtype=torch.float32, device="cuda"),
+        "counts": torch.empty(E, dtype=torch.int32, device="cuda"),
+        "offsets": torch.empty(E + 1, dtype=torch.int32, device="cuda"),
+        "perm": torch.empty(T * K, dtype=torch.int32, device="cuda"),
+        "inv": torch.empty(T * K, dtype=torch.int32, device="cuda"),
+        "logits": torch.empty((T, E), dtype=torch.float32, device="cuda"),
+    }
+    y = torch.full_like(xd, float("nan"))
+    M.moe_layer_forward(d, L.weights(M), xd, y, M.make_routing(**r), ws)
+    torch.cuda.synchronize()
+    assert M.moe_check_status(ws) == 0
+    mask = torch.empty(E, dtype=torch.uint8, device="cuda")
+    st = M.moe_expert_stats(d, r["counts"], mask, ws)
+
+    tokens = None if sample is None else mi.sample_tokens(T, sample, wl.seed + T).numpy()
+    ref = oracle.moe_layer_forward(mi.to_f64(x), L.wr64, L.bias, L.w1_64, L.w2_64, L.ws1_64,
+                                   L.ws2_64, K, tokens=tokens)
+    g = {k: to_np(v) for k, v in r.items()}
+    uniq, _, _ = compare_routing(wl, g["logits"], g["topk_idx"], g["topk_w"], ref["logits"], L.bias)
+    if uniq.all():
+        for k in ("counts", "offsets", "perm", "inv"):
+            assert (g[k] == ref[k]).all(), k
+        stats_equal(st, oracle.load_stats(ref["counts"], T, K))
+        assert (to_np(mask) == oracle.load_stats(ref["counts"], T, K)["straggler_mask"]).all()
+    else:
+        check_dispatch_valid(g["topk_idx"], g["counts"], g["offsets"], g["perm"], g["inv"], E)
+        stats_equal(st, oracle.load_stats(g["counts"], T, K))
+    tok = ref["tokens"]
+    keep = uniq[tok]
+    yg = to_np(y)[tok]
+    assert not np.isnan(to_np(y)).any(), "an output element was not written"
+    err = rel_max_err(yg[keep], ref["y"][keep])
+    assert err <= y_tol(wl), f"max |y - y_ref| = {err:.3e} x RMS"
+    return err, int((~uniq).sum())
+
+
+@pytest.mark.parametrize("key,T", FULL_POINTS)
+def test_layer_all_tokens(M, key, T):
+    run_and_check(M, layer(key), T)
+
+
+@pytest.mark.parametrize("key,T,n", SAMPLED_POINTS)
+def test_layer_sampled_tokens(M, key, T, n):
+    run_and_check(M, layer(key), T, sample=n)
+
+
+def test_layer_is_deterministic_and_writes_every_output(M):
+    L = layer("c1")
+    T = 64
+    d = L.desc(M, T)
+    ws = M.alloc_workspace(d)
+    x = mi.draw_x(L.wl, T).cuda()
+    ys = []
+    for fill in (float("nan"), 12345.0):
+        y = torch.full_like(x, fill)
+        M.moe_layer_forward(d, L.weights(M), x, y, None, ws)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1])
+
+
+def test_layer_ignores_stale_workspace_contents(M):
+    L = layer("c1")
+    T = 64
+    d = L.desc(M, T)
+    ws = M.alloc_workspace(d)
+    x = mi.draw_x(L.wl, T).cuda()
+    y0 = torch.empty_like(x)
+    M.moe_layer_forward(d, L.weights(M), x, y0, None, ws)
+    ws[256:].fill_(0xA5)                      # poison everything past the control header
+    y1 = torch.empty_like(x)
+    M.moe_layer_forward(d, L.weights(M), x, y1, None, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+
+
+@pytest.mark.parametrize("dtype,E,K,Ds", [("f32", 1, 1, 0), ("bf16", 1, 1, 128), ("f32", 6, 6, 0),
+                                          ("bf16", 16, 16, 0), ("bf16", 64, 4, 256)])
+def test_layer_edge_shapes(M, dtype, E, K, Ds):
+    H, D = (128, 256) if dtype == "bf16" else (64, 96)
+    wl = mi.Workload("edge", "edge case", dtype, H, E, K, D, Ds, (1, 13, 130), 11, zipf_s=1.2)
+    L = DeviceLayer(wl)
+    for T in wl.Ts:
+        run_and_check(M, L, T)
+
+
+def test_layer_empty_batch_is_a_no_op(M):
+    L = layer("c1")
+    d = L.desc(M, 0)
+    ws = M.alloc_workspace(d)
+    M.moe_layer_forward(d, L.weights(M), None, None, None, ws)
+    torch.cuda.synchronize()
+
+
+def test_workspace_too_small_is_rejected(M):
+    L = layer("c1")
+    d = L.desc(M, 64)
+    small = torch.zeros(M.moe_workspace_size(d) - 256, dtype=torch.uint8, device="cuda")
+    x = mi.draw_x(L.wl, 64).cuda()
+    with pytest.raises(M.MoEError) as ei:
+        M.moe_layer_forward(d, L.weights(M), x, torch.empty_like(x), None, small)
+    assert ei.value.status == 3
