@@ -190,6 +190,9 @@ def moe_layer_forward_profiled(desc, weights: MoELayerWeights, x, y, routing: Op
                                ws, events, stream=None):
     """moe_layer_forward recording torch.cuda.Event objects (6, timing-enabled)
     between its stages on the launching stream."""
+    for e in events:                 # torch creates the CUDA event on its first record
+        if not e.cuda_event:
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     _check(lib.moe_layer_forward_profiled(ctypes.byref(desc), ctypes.byref(weights), _p(x), _p(y),
                                           ctypes.byref(routing) if routing is not None else None,

@@ -51,8 +51,8 @@ WsLayout workspace_layout(const moe_layer_desc& d) {
   L.xp = take(d.dtype == MOE_BF16 ? es * TK * H : 0);
   L.hm = take(es * TK * D);
   L.hs = take(es * T * Ds);
-  L.yr = take(es * TK * H);
-  L.ys = take(es * T * H * (Ds ? 1 : 0));
+  L.yr = take(sizeof(float) * TK * H);   // expert outputs are fp32
+  L.ys = take(sizeof(float) * T * H * (Ds ? 1 : 0));
   L.stats = take(sizeof(moe_stats) + E);
   L.total = o;
   return L;
@@ -117,6 +117,23 @@ static moe_status run_grouped_ffn(const moe_layer_desc& d, const WsLayout& L, ch
   void* hm = ws + L.hm;
   void* hs = ws + L.hs;
   const bool shared = d.Ds > 0;
+  if (d.dtype == MOE_BF16) {
+    // Tensor-core path: the dispatched activation rows are in ws + L.xp.
+    const uint64_t TK = (uint64_t)d.T * d.K;
+    TcProblem r1{ws + L.xp, TK, w1, (uint64_t)d.E * d.D, d.D, d.H, hm, d.D, false};
+    TcProblem s1{x, (uint64_t)d.T, ws1, (uint64_t)d.Ds, d.Ds, d.H, hs, d.Ds, false};
+    TcProblem r2{hm, TK, w2, (uint64_t)d.E * d.H, d.H, d.D, y_rows, d.H, true};
+    TcProblem s2{hs, (uint64_t)d.T, ws2, (uint64_t)d.H, d.H, d.Ds, y_shared, d.H, true};
+    if (!shared) s1 = s2 = TcProblem{};
+    MOE_CUDA_TRY(launch_grouped_gemm_tc(r1, s1, d.E, true,
+                                        reinterpret_cast<const Tile*>(ws + L.tiles_tc1),
+                                        &hdr->n_tiles[1], &hdr->status, num_sms(), st));
+    if (ev_after_gemm1) MOE_CUDA_TRY(cudaEventRecord(*ev_after_gemm1, st));
+    MOE_CUDA_TRY(launch_grouped_gemm_tc(r2, s2, d.E, false,
+                                        reinterpret_cast<const Tile*>(ws + L.tiles_tc2),
+                                        &hdr->n_tiles[2], &hdr->status, num_sms(), st));
+    return MOE_OK;
+  }
   SimtProblem r1{x, perm, d.K, w1, (size_t)d.D * d.H, hm, d.H, d.D};
   SimtProblem s1{x, nullptr, 1, ws1, 0, hs, d.H, d.Ds};
   SimtProblem r2{hm, nullptr, 1, w2, (size_t)d.H * d.D, y_rows, d.D, d.H};
@@ -200,7 +217,9 @@ moe_status moe_grouped_ffn(const moe_layer_desc* desc, const void* x, const int3
   const WsLayout L = workspace_layout(d);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
-  MOE_CUDA_TRY(launch_tiles_from_offsets(d, L, w, offsets, false, st));
+  const bool tc = d.dtype == MOE_BF16;
+  MOE_CUDA_TRY(launch_tiles_from_offsets(d, L, w, offsets, tc, st));
+  if (tc) MOE_CUDA_TRY(launch_gather_rows(d, x, perm, w + L.xp, num_sms(), st));
   return run_grouped_ffn(d, L, w, x, perm, w1, w2, ws1, ws2, y_rows, y_shared, st);
 }
 
@@ -254,7 +273,9 @@ static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer
   MOE_CUDA_TRY(launch_gate_logits(d, x, W.w_router, logits, st));
   MOE_CUDA_TRY(launch_topk_select(d, logits, W.expert_bias, idx, tw, st));
   MOE_CUDA_TRY(mark(1));
-  MOE_CUDA_TRY(launch_dispatch(d, L, w, idx, counts, offsets, perm, inv, false, st));
+  const bool tc = d.dtype == MOE_BF16;
+  MOE_CUDA_TRY(launch_dispatch(d, L, w, idx, counts, offsets, perm, inv, tc, st));
+  if (tc) MOE_CUDA_TRY(launch_gather_rows(d, x, perm, w + L.xp, num_sms(), st));
   MOE_CUDA_TRY(mark(2));
   MOE_TRY(run_grouped_ffn(d, L, w, x, perm, W.w1, W.w2, W.ws1, W.ws2, yr, ys, st,
                           ev ? ev + 3 : nullptr));

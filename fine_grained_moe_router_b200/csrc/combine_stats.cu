@@ -54,13 +54,16 @@ struct CVec<float> {
   }
 };
 
+// Expert outputs are fp32; each thread sums V::N consecutive columns of one
+// token and rounds once to the layer dtype T.
 template <typename T>
-__global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_rows,
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_rows,
                                                       const float* __restrict__ w,
                                                       const int32_t* __restrict__ inv,
-                                                      const T* __restrict__ y_shared,
+                                                      const float* __restrict__ y_shared,
                                                       T* __restrict__ y, int T_, int H, int K) {
   using V = CVec<T>;
+  using F = CVec<float>;
   const int t = blockIdx.x;
   const int h = (blockIdx.y * blockDim.x + threadIdx.x) * V::N;
   if (t >= T_ || h >= H) return;
@@ -70,16 +73,24 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_ro
   for (int k = 0; k < K; ++k) {
     const int row = inv[(size_t)t * K + k];
     const float wk = w[(size_t)t * K + k];
-    float v[V::N];
-    V::load(y_rows + (size_t)row * H + h, v);
+    const float* src = y_rows + (size_t)row * H + h;
 #pragma unroll
-    for (int i = 0; i < V::N; ++i) acc[i] = fmaf(wk, v[i], acc[i]);
+    for (int q = 0; q < V::N; q += F::N) {
+      float v[F::N];
+      F::load(src + q, v);
+#pragma unroll
+      for (int i = 0; i < F::N; ++i) acc[q + i] = fmaf(wk, v[i], acc[q + i]);
+    }
   }
   if (y_shared) {
-    float v[V::N];
-    V::load(y_shared + (size_t)t * H + h, v);
+    const float* src = y_shared + (size_t)t * H + h;
 #pragma unroll
-    for (int i = 0; i < V::N; ++i) acc[i] += v[i];
+    for (int q = 0; q < V::N; q += F::N) {
+      float v[F::N];
+      F::load(src + q, v);
+#pragma unroll
+      for (int i = 0; i < F::N; ++i) acc[q + i] += v[i];
+    }
   }
   V::store(y + (size_t)t * H + h, acc);
 }
@@ -93,8 +104,7 @@ cudaError_t launch_combine(const moe_layer_desc& d, const void* y_rows, const fl
   count_launch();
   if (d.dtype == MOE_BF16)
     combine_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
-        (const __nv_bfloat16*)y_rows, w, inv, (const __nv_bfloat16*)y_shared,
-        (__nv_bfloat16*)y, d.T, d.H, d.K);
+        (const float*)y_rows, w, inv, (const float*)y_shared, (__nv_bfloat16*)y, d.T, d.H, d.K);
   else
     combine_kernel<float><<<grid, threads, 0, st>>>((const float*)y_rows, w, inv,
                                                     (const float*)y_shared, (float*)y, d.T, d.H,

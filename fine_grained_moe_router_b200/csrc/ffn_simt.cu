@@ -94,27 +94,35 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt(const Tile* __restrict_
   }
 }
 
-template <typename T, bool kGelu>
+template <typename TIn, typename TOut, bool kGelu>
 static cudaError_t launch_simt_t(const SimtProblem& routed, const SimtProblem& shared, int E,
                                  const Tile* tiles, const int* n_tiles, int max_tiles, int max_n,
                                  cudaStream_t st) {
   if (max_tiles <= 0) return cudaSuccess;
   dim3 grid(max_tiles, (max_n + kBN - 1) / kBN);
   count_launch();
-  grouped_gemm_simt<T, T, kGelu><<<grid, 256, 0, st>>>(tiles, n_tiles, routed, shared, E);
+  grouped_gemm_simt<TIn, TOut, kGelu><<<grid, 256, 0, st>>>(tiles, n_tiles, routed, shared, E);
   return cudaGetLastError();
 }
 
-cudaError_t launch_grouped_gemm_simt(int dtype, bool gelu, const SimtProblem& routed,
+// First layer: output in the input dtype with GeLU; second layer: fp32
+// output without activation.
+cudaError_t launch_grouped_gemm_simt(int dtype, bool first_layer, const SimtProblem& routed,
                                      const SimtProblem& shared, int E, const Tile* tiles,
                                      const int* n_tiles, int max_tiles, int max_n,
                                      cudaStream_t st) {
   if (dtype == MOE_BF16) {
-    return gelu ? launch_simt_t<__nv_bfloat16, true>(routed, shared, E, tiles, n_tiles, max_tiles, max_n, st)
-                : launch_simt_t<__nv_bfloat16, false>(routed, shared, E, tiles, n_tiles, max_tiles, max_n, st);
+    return first_layer
+               ? launch_simt_t<__nv_bfloat16, __nv_bfloat16, true>(routed, shared, E, tiles,
+                                                                   n_tiles, max_tiles, max_n, st)
+               : launch_simt_t<__nv_bfloat16, float, false>(routed, shared, E, tiles, n_tiles,
+                                                            max_tiles, max_n, st);
   }
-  return gelu ? launch_simt_t<float, true>(routed, shared, E, tiles, n_tiles, max_tiles, max_n, st)
-              : launch_simt_t<float, false>(routed, shared, E, tiles, n_tiles, max_tiles, max_n, st);
+  return first_layer
+             ? launch_simt_t<float, float, true>(routed, shared, E, tiles, n_tiles, max_tiles,
+                                                 max_n, st)
+             : launch_simt_t<float, float, false>(routed, shared, E, tiles, n_tiles, max_tiles,
+                                                  max_n, st);
 }
 
 }  // namespace moe

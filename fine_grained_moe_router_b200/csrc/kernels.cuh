@@ -17,6 +17,25 @@ struct SimtProblem {
   int N;                   // output columns
 };
 
+// One side (routed experts or shared expert) of a grouped GEMM on the tensor
+// cores. act [act_rows, kd] and w [w_rows, kd] are bf16 row-major; the
+// group g occupies weight rows [g * m_rows, (g + 1) * m_rows).
+struct TcProblem {
+  const void* act;
+  uint64_t act_rows;
+  const void* w;
+  uint64_t w_rows;
+  int m_rows;
+  int kd;
+  void* out;               // [*, ld], bf16 (first layer) or fp32 (out_f32)
+  int ld;
+  bool out_f32;
+};
+
+cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& shared, int E,
+                                   bool gelu, const Tile* tiles, const int* n_tiles,
+                                   uint32_t* status, int num_sms, cudaStream_t st);
+
 cudaError_t launch_gate_logits(const moe_layer_desc& d, const void* x, const void* wr,
                                float* logits, cudaStream_t st);
 cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, const float* bias,

@@ -29,9 +29,10 @@
  *    so every GEMM operand is contiguous along its reduction dimension:
  *      x [T, H], W_r [E, H], W1 [E, D, H], W2 [E, H, D], Ws1 [Ds, H],
  *      Ws2 [H, Ds], y [T, H].
- *    Element type of x / weights / y / y_rows / y_shared is desc->dtype
- *    (MOE_F32 or MOE_BF16). Logits, top-K weights and the bias are fp32;
- *    indices, counts, offsets, perm and inv are int32.
+ *    Element type of x / weights / y is desc->dtype (MOE_F32 or MOE_BF16).
+ *    The per-copy expert outputs y_rows / y_shared are always fp32, so the
+ *    combine rounds the layer output exactly once. Logits, top-K weights and
+ *    the bias are fp32; indices, counts, offsets, perm and inv are int32.
  *  - Device pointers must be 16-byte aligned.
  *  - The caller owns every buffer, including the workspace; the library
  *    never allocates device memory. The workspace must hold
@@ -159,16 +160,19 @@ moe_status moe_dispatch(const moe_layer_desc* desc, const int32_t* topk_idx, int
  * "Kimi K3 fine-grained MoE ...", section "通信-计算时间比的代数拐点"
  * (2*H*D multiply-adds per copy and layer).
  *   y_rows[row, :] = GeLU(x[perm[row] / K] W1[e]^T) W2[e]^T for every row of
- *   expert e's segment offsets[e] .. offsets[e+1]-1; y_rows [T*K, H].
- *   y_shared [T, H] = GeLU(x Ws1^T) Ws2^T when Ds > 0 (else may be NULL).
- *   GeLU is the exact erf form. Accumulation is fp32. */
+ *   expert e's segment offsets[e] .. offsets[e+1]-1; y_rows [T*K, H] fp32.
+ *   y_shared [T, H] fp32 = GeLU(x Ws1^T) Ws2^T when Ds > 0 (else may be NULL).
+ *   GeLU is the exact erf form. Accumulation is fp32; the GeLU output that
+ *   feeds the second Linear is rounded to desc->dtype (the tensor-core
+ *   operand type for bf16 layers). */
 moe_status moe_grouped_ffn(const moe_layer_desc* desc, const void* x, const int32_t* perm,
                            const int32_t* offsets, const void* w1, const void* w2,
                            const void* ws1, const void* ws2, void* y_rows, void* y_shared,
                            void* ws, size_t ws_bytes, moe_stream stream);
 
 /* Combine: y[t] = sum_{k=0}^{K-1} topk_w[t,k] * y_rows[inv[t*K+k]] (+ y_shared[t]),
- * summed in fp32 in that order, rounded once to desc->dtype. No residual.
+ * y_rows / y_shared fp32, summed in fp32 in that order, rounded once to
+ * desc->dtype. No residual.
  * "Kimi K3 fine-grained MoE ...", section "物理通信拓扑" (combine phase);
  * "MoE architecture in production" §3.1 (scatter back to original order). */
 moe_status moe_combine(const moe_layer_desc* desc, const void* y_rows, const float* topk_w,

@@ -103,8 +103,8 @@ def test_grouped_ffn_matches_oracle(M, dtype, T, H, E, K, D, Ds):
     d = M.make_desc(T, H, E, K, D, Ds, M.MOE_F32 if dtype == "f32" else M.MOE_BF16)
     ws = M.alloc_workspace(d)
     dev = lambda t: t.cuda() if t is not None else None
-    y_rows = torch.empty((T * K, H), dtype=tdt, device="cuda")
-    y_sh = torch.empty((T, H), dtype=tdt, device="cuda") if Ds else None
+    y_rows = torch.empty((T * K, H), dtype=torch.float32, device="cuda")   # expert outputs: fp32
+    y_sh = torch.empty((T, H), dtype=torch.float32, device="cuda") if Ds else None
     M.moe_grouped_ffn(d, dev(x), torch.from_numpy(perm_np).cuda(), torch.from_numpy(off_np).cuda(),
                       dev(w1), dev(w2), dev(ws1), dev(ws2), y_rows, y_sh, ws)
     f64 = lambda t: t.double().numpy() if t is not None else None
@@ -121,13 +121,13 @@ def test_grouped_ffn_matches_oracle(M, dtype, T, H, E, K, D, Ds):
 def test_combine_matches_oracle(M, dtype, T, H, K, shared):
     rng = np.random.default_rng(T * H + K)
     tdt = torch.float32 if dtype == "f32" else torch.bfloat16
-    rows = torch.from_numpy(rng.normal(size=(T * K, H)).astype(np.float32)).to(tdt)
+    rows = torch.from_numpy(rng.normal(size=(T * K, H)).astype(np.float32))   # fp32 expert outputs
     w = rng.random(size=(T, K)).astype(np.float32)
     w /= w.sum(1, keepdims=True)
     perm = rng.permutation(T * K).astype(np.int32)
     inv = np.empty_like(perm)
     inv[perm] = np.arange(T * K, dtype=np.int32)
-    sh = torch.from_numpy(rng.normal(size=(T, H)).astype(np.float32)).to(tdt) if shared else None
+    sh = torch.from_numpy(rng.normal(size=(T, H)).astype(np.float32)) if shared else None
     d = M.make_desc(T, H, 8, K, 128, 128 if shared else 0, M.MOE_F32 if dtype == "f32" else M.MOE_BF16)
     y = torch.empty((T, H), dtype=tdt, device="cuda")
     M.moe_combine(d, rows.cuda(), torch.from_numpy(w).cuda(), torch.from_numpy(inv).cuda(),
