@@ -24,7 +24,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_router_topk", "moe_topk_from_logits", "moe_dispatch",
     "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
     "moe_expert_stats",
-    "moe_check_status", "moe_status_string", "moe_kernel_launch_count",
+    "moe_check_status", "moe_status_string", "moe_kernel_launch_count", "moe_dispatch_noalloc",
 )
 
 
@@ -80,6 +80,7 @@ def _load() -> ctypes.CDLL:
         "moe_check_status": (ctypes.c_int, [P, S, P]),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_kernel_launch_count": (ctypes.c_uint64, []),
+        "moe_dispatch_noalloc": (ctypes.c_int, [D, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -150,6 +151,14 @@ def moe_dispatch(desc, topk_idx, counts, offsets, perm, inv, ws, stream=None):
     _check(lib.moe_dispatch(ctypes.byref(desc), _p(topk_idx), _p(counts), _p(offsets), _p(perm),
                             _p(inv), _p(ws), ws.numel() if ws is not None else 0, _stream(stream)),
            "moe_dispatch")
+
+
+def moe_dispatch_noalloc(desc, topk_idx, counts, offsets, perm, inv, stream=None):
+    """moe_dispatch without a workspace, for callers that cannot allocate device
+    memory: its scratch is a fixed array inside libmoe (T*K <= 65536). Calls that
+    overlap on the GPU share that array and race."""
+    _check(lib.moe_dispatch_noalloc(ctypes.byref(desc), _p(topk_idx), _p(counts), _p(offsets),
+                                    _p(perm), _p(inv), _stream(stream)), "moe_dispatch_noalloc")
 
 
 def moe_grouped_ffn(desc, x, perm, offsets, w1, w2, ws1, ws2, y_rows, y_shared, ws, stream=None):

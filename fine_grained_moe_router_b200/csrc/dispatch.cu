@@ -285,6 +285,31 @@ cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws
   return cudaGetLastError();
 }
 
+// The same three dispatch kernels with caller-provided scratch: hist and base
+// hold n_chunks * E ints each; no tile lists are written.
+cudaError_t launch_dispatch_scratch(const moe_layer_desc& d, int n_chunks, int32_t* hist,
+                                   int32_t* base, WsHeader* hdr, const int32_t* idx,
+                                   int32_t* counts, int32_t* offsets, int32_t* perm,
+                                   int32_t* inv, cudaStream_t st) {
+  const int TK = d.T * d.K;
+  if (TK > 0) {
+    count_launch();
+    chunk_histogram<<<n_chunks, 256, 0, st>>>(idx, TK, d.E, hist, &hdr->status);
+  } else {
+    cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(int32_t) * (size_t)n_chunks * d.E, st);
+    if (e != cudaSuccess) return e;
+  }
+  TileSpec ts{};
+  count_launch();
+  scan_and_tiles<<<1, 1024, 0, st>>>(hist, n_chunks, d.E, d.T, d.Ds > 0 ? 1 : 0, counts, offsets,
+                                     base, ts, hdr);
+  if (TK > 0) {
+    count_launch();
+    chunk_scatter<<<n_chunks, 256, 0, st>>>(idx, TK, d.E, base, perm, inv);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_tiles_from_offsets(const moe_layer_desc& d, const WsLayout& L, char* ws,
                                       const int32_t* offsets, bool tc_tiles, cudaStream_t st) {
   const TileSpec ts = make_tile_spec(d, L, ws, tc_tiles);

@@ -43,6 +43,10 @@ cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, con
 cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws,
                             const int32_t* idx, int32_t* counts, int32_t* offsets,
                             int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st);
+cudaError_t launch_dispatch_scratch(const moe_layer_desc& d, int n_chunks, int32_t* hist,
+                                   int32_t* base, WsHeader* hdr, const int32_t* idx,
+                                   int32_t* counts, int32_t* offsets, int32_t* perm,
+                                   int32_t* inv, cudaStream_t st);
 cudaError_t launch_tiles_from_offsets(const moe_layer_desc& d, const WsLayout& L, char* ws,
                                       const int32_t* offsets, bool tc_tiles, cudaStream_t st);
 cudaError_t launch_gather_rows(const moe_layer_desc& d, const void* x, const int32_t* perm,

@@ -155,6 +155,25 @@ moe_status moe_dispatch(const moe_layer_desc* desc, const int32_t* topk_idx, int
                         int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
                         size_t ws_bytes, moe_stream stream);
 
+/* moe_dispatch for callers that cannot allocate device memory (a plugin
+ * whose host runtime owns every allocation, a server whose memory pool is
+ * fully reserved after warm-up, a latency-critical path that cannot afford
+ * cudaMalloc's implicit synchronisation). The pages have no counterpart of
+ * this call; it exists only for such callers.
+ * Same arguments and results as moe_dispatch, without a workspace: the
+ * scratch (per-chunk histograms) lives in a 128.25 KiB array of device
+ * memory inside the library, held by every GPU that loads it until the
+ * process exits. Limit: T*K <= 65536 (plus the usual E <= 512, K <= 16);
+ * larger batches return MOE_ERR_UNSUPPORTED without launching. The first
+ * call on a device looks up the array's device address (once per device,
+ * with that device current): make that first call before any stream
+ * capture. All calls share the array, so calls that overlap on the GPU race.
+ * Out-of-range indices are skipped (counts then sum to less than T*K) and
+ * not reported. Allocates nothing. */
+moe_status moe_dispatch_noalloc(const moe_layer_desc* desc, const int32_t* topk_idx,
+                                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                                moe_stream stream);
+
 /* Grouped expert FFN over the dispatched rows, plus the shared expert.
  * "MoE architecture in production" §3.1 (experts of Linear, GeLU, Linear);
  * "Kimi K3 fine-grained MoE ...", section "通信-计算时间比的代数拐点"
