@@ -211,11 +211,6 @@ def time_oracle(wl, inp, T, n_tokens, seed):
     return time.perf_counter() - t0, len(tokens)
 
 
-def default_sample(wl, T):
-    # about 10-30 s of fp64 work on the host for the cpu_baseline leg
-    return min(T, 256 if wl.E <= 16 else 128)
-
-
 # ------------------------------------------------------------ reference ---
 def run_reference(args, wl, T):
     rank, world, _ = dist_info()
@@ -436,9 +431,13 @@ def sweep(M, wl, dev, T_main, peaks, all_workloads):
     return out
 
 
-def cpu_baseline(wl, host, x, T):
+def cpu_baseline(wl, host, x, T, target_s=15.0):
+    """The oracle on the host cores: a short calibration run, then a sample
+    sized to about target_s seconds (the whole batch if that is less)."""
     inp = widen_all(oracle_inputs(wl, host, x))
-    n = default_sample(wl, T)
+    n0 = min(T, 64)
+    dt0, _ = time_oracle(wl, inp, T, n0, seed=6)
+    n = T if dt0 * T / n0 <= 2 * target_s else max(n0, int(n0 * target_s / max(dt0, 1e-3)))
     dt, n_done = time_oracle(wl, inp, T, n, seed=7)
     return {"value": n_done / dt, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
             "sample": f"routing of all {T} tokens + expert FFNs of {n_done} seeded sample tokens "

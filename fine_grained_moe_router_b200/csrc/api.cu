@@ -16,6 +16,48 @@ size_t dtype_size(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
 
 static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// Reduction splits for the tensor-core GEMMs. A decode-sized step has too
+// few (128-row x all-K) tiles to give every one of the 148 SMs a share of
+// the weight stream; splitting the reduction multiplies the tiles. The
+// choice depends on the shape only (so the workspace size does too):
+// about kTargetTiles tiles, at least 2 (router) or 4 (expert GEMM) reduction
+// blocks per split, and no empty split.
+static int split_count(long long tiles, int kb, int want_tiles, int min_kb) {
+  if (tiles <= 0 || tiles >= want_tiles) return 1;
+  int sp = (int)((want_tiles + tiles - 1) / tiles);
+  sp = std::min(sp, std::max(1, kb / min_kb));
+  sp = std::max(1, std::min(sp, kMaxSplits));
+  const int per = (kb + sp - 1) / sp;
+  return (kb + per - 1) / per;
+}
+
+Splits choose_splits(const moe_layer_desc& d) {
+  Splits s{1, 1, 1};
+  if (d.dtype != MOE_BF16 || d.T == 0) return s;
+  constexpr int kTargetTiles = 296;   // two per SM
+  const long long T = d.T, TK = (long long)d.T * d.K;
+  const long long row_tiles = (T + kTcRows - 1) / kTcRows;
+  s.router = std::min(16, split_count(row_tiles * ((d.E + 127) / 128), d.H / 64,
+                                      kTargetTiles / 2, 2));
+  {  // no empty split after the cap
+    const int kb = d.H / 64, per = (kb + s.router - 1) / s.router;
+    s.router = (kb + per - 1) / per;
+  }
+  // GEMM2: each touched expert has at least one row tile; a decode step
+  // touches min(E, T*K) experts.
+  const int mt2 = d.H / 128;
+  const long long r_tiles = std::max(std::min<long long>(d.E, TK), (TK + kTcRows - 1) / kTcRows) * mt2;
+  const long long s_tiles = d.Ds ? row_tiles * mt2 : 0;
+  if (r_tiles + s_tiles < kTargetTiles) {
+    const int kbr = d.D / 64, kbs = d.Ds / 64;
+    const long long total_kb = r_tiles * kbr + s_tiles * kbs;
+    const int per = (int)std::max<long long>(4, (total_kb + kTargetTiles - 1) / kTargetTiles);
+    s.gemm2_routed = split_count(1, kbr, (kbr + per - 1) / per, 4);
+    if (d.Ds) s.gemm2_shared = split_count(1, kbs, (kbs + per - 1) / per, 4);
+  }
+  return s;
+}
+
 WsLayout workspace_layout(const moe_layer_desc& d) {
   WsLayout L{};
   const size_t T = d.T, K = d.K, E = d.E, H = d.H, D = d.D, Ds = d.Ds;
@@ -27,8 +69,10 @@ WsLayout workspace_layout(const moe_layer_desc& d) {
                            (Ds ? (T + kSimtRows - 1) / kSimtRows : 0));
   const size_t rt_routed = (TK + kTcRows - 1) / kTcRows + rows_bound;
   const size_t rt_shared = Ds ? (T + kTcRows - 1) / kTcRows : 0;
+  L.sp = choose_splits(d);
   L.max_tiles_tc1 = (int)(rt_routed * (D / 128) + rt_shared * (Ds / 128));
-  L.max_tiles_tc2 = (int)((rt_routed + rt_shared) * (H / 128));
+  L.max_tiles_tc2 =
+      (int)((rt_routed * L.sp.gemm2_routed + rt_shared * L.sp.gemm2_shared) * (H / 128));
   size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -48,11 +92,13 @@ WsLayout workspace_layout(const moe_layer_desc& d) {
   L.perm = take(sizeof(int32_t) * TK);
   L.inv = take(sizeof(int32_t) * TK);
   L.logits = take(sizeof(float) * T * E);
+  L.logits_part = take(d.dtype == MOE_BF16 ? sizeof(float) * T * E * L.sp.router : 0);
   L.xp = take(d.dtype == MOE_BF16 ? es * TK * H : 0);
   L.hm = take(es * TK * D);
   L.hs = take(es * T * Ds);
-  L.yr = take(sizeof(float) * TK * H);   // expert outputs are fp32
-  L.ys = take(sizeof(float) * T * H * (Ds ? 1 : 0));
+  // expert outputs are fp32, one copy per reduction split of the second GEMM
+  L.yr = take(sizeof(float) * TK * H * L.sp.gemm2_routed);
+  L.ys = take(sizeof(float) * T * H * (Ds ? L.sp.gemm2_shared : 0));
   L.stats = take(sizeof(moe_stats) + E);
   L.total = o;
   return L;
@@ -110,7 +156,7 @@ static int num_sms() {
 static moe_status run_grouped_ffn(const moe_layer_desc& d, const WsLayout& L, char* ws,
                                   const void* x, const int32_t* perm, const void* w1,
                                   const void* w2, const void* ws1, const void* ws2, void* y_rows,
-                                  void* y_shared, cudaStream_t st,
+                                  void* y_shared, cudaStream_t st, bool split,
                                   cudaEvent_t const* ev_after_gemm1 = nullptr) {
   if (d.T == 0) return MOE_OK;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
@@ -120,18 +166,41 @@ static moe_status run_grouped_ffn(const moe_layer_desc& d, const WsLayout& L, ch
   if (d.dtype == MOE_BF16) {
     // Tensor-core path: the dispatched activation rows are in ws + L.xp.
     const uint64_t TK = (uint64_t)d.T * d.K;
-    TcProblem r1{ws + L.xp, TK, w1, (uint64_t)d.E * d.D, d.D, d.H, hm, d.D, false};
-    TcProblem s1{x, (uint64_t)d.T, ws1, (uint64_t)d.Ds, d.Ds, d.H, hs, d.Ds, false};
-    TcProblem r2{hm, TK, w2, (uint64_t)d.E * d.H, d.H, d.D, y_rows, d.H, true};
-    TcProblem s2{hs, (uint64_t)d.T, ws2, (uint64_t)d.H, d.H, d.Ds, y_shared, d.H, true};
-    if (!shared) s1 = s2 = TcProblem{};
+    auto problem = [](const void* act, uint64_t act_rows, const void* w, uint64_t w_rows,
+                      int m_rows, int kd, void* out, int ld, bool out_f32, int splits,
+                      long long split_stride) {
+      TcProblem p{};
+      p.act = act;
+      p.act_rows = act_rows;
+      p.w = w;
+      p.w_rows = w_rows;
+      p.m_rows = m_rows;
+      p.kd = kd;
+      p.out = out;
+      p.ld = ld;
+      p.out_f32 = out_f32;
+      p.splits = splits;
+      p.split_stride = split_stride;
+      p.m_valid = m_rows;
+      return p;
+    };
+    const int sp_r = split ? L.sp.gemm2_routed : 1, sp_s = split ? L.sp.gemm2_shared : 1;
+    TcProblem r1 = problem(ws + L.xp, TK, w1, (uint64_t)d.E * d.D, d.D, d.H, hm, d.D, false, 1, 0);
+    TcProblem r2 = problem(hm, TK, w2, (uint64_t)d.E * d.H, d.H, d.D, y_rows, d.H, true, sp_r,
+                           (long long)TK * d.H);
+    TcProblem s1{}, s2{};
+    if (shared) {
+      s1 = problem(x, (uint64_t)d.T, ws1, (uint64_t)d.Ds, d.Ds, d.H, hs, d.Ds, false, 1, 0);
+      s2 = problem(hs, (uint64_t)d.T, ws2, (uint64_t)d.H, d.H, d.Ds, y_shared, d.H, true, sp_s,
+                   (long long)d.T * d.H);
+    }
     MOE_CUDA_TRY(launch_grouped_gemm_tc(r1, s1, d.E, true,
                                         reinterpret_cast<const Tile*>(ws + L.tiles_tc1),
-                                        &hdr->n_tiles[1], &hdr->status, num_sms(), st));
+                                        &hdr->n_tiles[1], nullptr, &hdr->status, num_sms(), st));
     if (ev_after_gemm1) MOE_CUDA_TRY(cudaEventRecord(*ev_after_gemm1, st));
     MOE_CUDA_TRY(launch_grouped_gemm_tc(r2, s2, d.E, false,
                                         reinterpret_cast<const Tile*>(ws + L.tiles_tc2),
-                                        &hdr->n_tiles[2], &hdr->status, num_sms(), st));
+                                        &hdr->n_tiles[2], nullptr, &hdr->status, num_sms(), st));
     return MOE_OK;
   }
   SimtProblem r1{x, perm, d.K, w1, (size_t)d.D * d.H, hm, d.H, d.D};
@@ -144,6 +213,26 @@ static moe_status run_grouped_ffn(const moe_layer_desc& d, const WsLayout& L, ch
   if (ev_after_gemm1) MOE_CUDA_TRY(cudaEventRecord(*ev_after_gemm1, st));
   MOE_CUDA_TRY(launch_grouped_gemm_simt(d.dtype, false, r2, s2, d.E, tiles, &hdr->n_tiles[0],
                                         L.max_tiles_simt, d.H, st));
+  return MOE_OK;
+}
+
+// Router: gate logits then selection. bf16 layers run the gate GEMM on the
+// tensor cores (partial sums per reduction split, added by the selection
+// kernel); fp32 layers on CUDA cores.
+static moe_status run_router(const moe_layer_desc& d, const WsLayout& L, char* ws,
+                             const void* x, const void* wr, const float* bias, int32_t* idx,
+                             float* tw, float* logits_out, cudaStream_t st) {
+  if (d.T == 0) return MOE_OK;
+  if (d.dtype == MOE_BF16) {
+    float* parts = reinterpret_cast<float*>(ws + L.logits_part);
+    MOE_CUDA_TRY(launch_gate_logits_tc(d, L, ws, x, wr, parts, num_sms(), st));
+    MOE_CUDA_TRY(launch_topk_select(d, parts, L.sp.router, (size_t)d.T * d.E, bias, idx, tw,
+                                    logits_out, st));
+  } else {
+    float* logits = logits_out ? logits_out : reinterpret_cast<float*>(ws + L.logits);
+    MOE_CUDA_TRY(launch_gate_logits(d, x, wr, logits, st));
+    MOE_CUDA_TRY(launch_topk_select(d, logits, 1, 0, bias, idx, tw, nullptr, st));
+  }
   return MOE_OK;
 }
 
@@ -170,11 +259,8 @@ moe_status moe_router_topk(const moe_layer_desc* desc, const void* x, const void
   if (logits_or_null && !aligned16(logits_or_null)) return MOE_ERR_INVALID_ARG;
   const WsLayout L = workspace_layout(d);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* logits = logits_or_null ? logits_or_null
-                                 : reinterpret_cast<float*>(static_cast<char*>(ws) + L.logits);
-  MOE_CUDA_TRY(launch_gate_logits(d, x, w_router, logits, st));
-  MOE_CUDA_TRY(launch_topk_select(d, logits, bias, topk_idx, topk_w, st));
-  return MOE_OK;
+  return run_router(d, L, static_cast<char*>(ws), x, w_router, bias, topk_idx, topk_w,
+                    logits_or_null, st);
 }
 
 moe_status moe_topk_from_logits(const moe_layer_desc* desc, const float* logits,
@@ -185,7 +271,7 @@ moe_status moe_topk_from_logits(const moe_layer_desc* desc, const float* logits,
   if (d.T == 0) return MOE_OK;
   MOE_TRY(check_ptrs({logits, topk_idx, topk_w}));
   if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
-  MOE_CUDA_TRY(launch_topk_select(d, logits, bias, topk_idx, topk_w,
+  MOE_CUDA_TRY(launch_topk_select(d, logits, 1, 0, bias, topk_idx, topk_w, nullptr,
                                   static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
@@ -220,7 +306,8 @@ moe_status moe_grouped_ffn(const moe_layer_desc* desc, const void* x, const int3
   const bool tc = d.dtype == MOE_BF16;
   MOE_CUDA_TRY(launch_tiles_from_offsets(d, L, w, offsets, tc, st));
   if (tc) MOE_CUDA_TRY(launch_gather_rows(d, x, perm, w + L.xp, num_sms(), st));
-  return run_grouped_ffn(d, L, w, x, perm, w1, w2, ws1, ws2, y_rows, y_shared, st);
+  return run_grouped_ffn(d, L, w, x, perm, w1, w2, ws1, ws2, y_rows, y_shared, st,
+                         /*split=*/false);
 }
 
 moe_status moe_combine(const moe_layer_desc* desc, const void* y_rows, const float* topk_w,
@@ -258,7 +345,6 @@ static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer
     if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
   const WsLayout L = workspace_layout(d);
   char* w = static_cast<char*>(ws);
-  float* logits = R.logits ? R.logits : reinterpret_cast<float*>(w + L.logits);
   int32_t* idx = R.topk_idx ? R.topk_idx : reinterpret_cast<int32_t*>(w + L.idx);
   float* tw = R.topk_w ? R.topk_w : reinterpret_cast<float*>(w + L.w);
   int32_t* counts = R.counts ? R.counts : reinterpret_cast<int32_t*>(w + L.counts);
@@ -270,17 +356,16 @@ static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer
   auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
 
   MOE_CUDA_TRY(mark(0));
-  MOE_CUDA_TRY(launch_gate_logits(d, x, W.w_router, logits, st));
-  MOE_CUDA_TRY(launch_topk_select(d, logits, W.expert_bias, idx, tw, st));
+  MOE_TRY(run_router(d, L, w, x, W.w_router, W.expert_bias, idx, tw, R.logits, st));
   MOE_CUDA_TRY(mark(1));
   const bool tc = d.dtype == MOE_BF16;
   MOE_CUDA_TRY(launch_dispatch(d, L, w, idx, counts, offsets, perm, inv, tc, st));
   if (tc) MOE_CUDA_TRY(launch_gather_rows(d, x, perm, w + L.xp, num_sms(), st));
   MOE_CUDA_TRY(mark(2));
   MOE_TRY(run_grouped_ffn(d, L, w, x, perm, W.w1, W.w2, W.ws1, W.ws2, yr, ys, st,
-                          ev ? ev + 3 : nullptr));
+                          /*split=*/true, ev ? ev + 3 : nullptr));
   MOE_CUDA_TRY(mark(4));
-  MOE_CUDA_TRY(launch_combine(d, yr, tw, inv, ys, y, st));
+  MOE_CUDA_TRY(launch_combine(d, yr, tw, inv, ys, y, st, L.sp.gemm2_routed, L.sp.gemm2_shared));
   MOE_CUDA_TRY(mark(5));
   return MOE_OK;
 }

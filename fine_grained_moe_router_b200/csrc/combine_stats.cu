@@ -16,6 +16,7 @@
 // may swap ranks without changing the sum, so no sort is needed.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -56,12 +57,35 @@ struct CVec<float> {
 
 // Expert outputs are fp32; each thread sums V::N consecutive columns of one
 // token and rounds once to the layer dtype T.
+// Sum of n_parts partial rows (reduction splits of the second expert GEMM),
+// added in split order.
+template <int N>
+__device__ __forceinline__ void load_parts(const float* src, int n_parts, size_t stride,
+                                           float* v) {
+  CVec<float>::load(src, v);
+  for (int p0 = 1; p0 < n_parts; p0 += 4) {   // 4 independent loads, then in-order adds
+    float u[4][4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (p0 + q < n_parts) CVec<float>::load(src + (p0 + q) * stride, u[q]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (p0 + q < n_parts)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = __fadd_rn(v[i], u[q][i]);
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_rows,
+                                                      int rows_parts, size_t rows_stride,
                                                       const float* __restrict__ w,
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ y_shared,
+                                                      int shared_parts, size_t shared_stride,
                                                       T* __restrict__ y, int T_, int H, int K) {
+  pdl_wait();
+  pdl_trigger();
   using V = CVec<T>;
   using F = CVec<float>;
   const int t = blockIdx.x;
@@ -77,7 +101,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 #pragma unroll
     for (int q = 0; q < V::N; q += F::N) {
       float v[F::N];
-      F::load(src + q, v);
+      load_parts<F::N>(src + q, rows_parts, rows_stride, v);
 #pragma unroll
       for (int i = 0; i < F::N; ++i) acc[q + i] = fmaf(wk, v[i], acc[q + i]);
     }
@@ -87,7 +111,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 #pragma unroll
     for (int q = 0; q < V::N; q += F::N) {
       float v[F::N];
-      F::load(src + q, v);
+      load_parts<F::N>(src + q, shared_parts, shared_stride, v);
 #pragma unroll
       for (int i = 0; i < F::N; ++i) acc[q + i] += v[i];
     }
@@ -96,20 +120,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 }
 
 cudaError_t launch_combine(const moe_layer_desc& d, const void* y_rows, const float* w,
-                           const int32_t* inv, const void* y_shared, void* y, cudaStream_t st) {
+                           const int32_t* inv, const void* y_shared, void* y, cudaStream_t st,
+                           int rows_parts, int shared_parts) {
   if (d.T == 0) return cudaSuccess;
   const int vec = (d.dtype == MOE_BF16) ? 8 : 4;
   const int threads = 128;
   dim3 grid(d.T, (d.H / vec + threads - 1) / threads);
-  count_launch();
+  const size_t rows_stride = (size_t)d.T * d.K * d.H, shared_stride = (size_t)d.T * d.H;
   if (d.dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
-        (const float*)y_rows, w, inv, (const float*)y_shared, (__nv_bfloat16*)y, d.T, d.H, d.K);
-  else
-    combine_kernel<float><<<grid, threads, 0, st>>>((const float*)y_rows, w, inv,
-                                                    (const float*)y_shared, (float*)y, d.T, d.H,
-                                                    d.K);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(threads), 0, st,
+                      (const float*)y_rows, rows_parts, rows_stride, w, inv,
+                      (const float*)y_shared, shared_parts, shared_stride, (__nv_bfloat16*)y,
+                      d.T, d.H, d.K);
+  return launch_pdl(combine_kernel<float>, grid, dim3(threads), 0, st, (const float*)y_rows,
+                    rows_parts, rows_stride, w, inv, (const float*)y_shared, shared_parts,
+                    shared_stride, (float*)y, d.T, d.H, d.K);
 }
 
 // ---------------------------------------------------------------------------
@@ -117,6 +142,8 @@ __global__ void __launch_bounds__(512) expert_stats_kernel(const int32_t* __rest
                                                            int E, long long TK, int capacity,
                                                            uint8_t* __restrict__ mask,
                                                            moe_stats* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int c[kMaxE];
   __shared__ long long red[6][16];
   const int j = threadIdx.x;

@@ -50,20 +50,35 @@ struct Tile {
   int32_t r0;
   int32_t n;
   int32_t m0;   // first output column (weight row) of the tile; used by the tensor-core path
+  int32_t ks;   // reduction split of the tile (tensor-core path), 0 when unsplit
+  int32_t pad[3];
+};
+
+// Reduction splits of the tensor-core GEMMs of one layer forward (chosen on
+// the host from the shape alone). A split s of a tile covers reduction blocks
+// [s * kb_per, (s + 1) * kb_per) and writes its own fp32 partial output; the
+// consumer kernel adds the partials in split order.
+struct Splits {
+  int router;        // gate GEMM
+  int gemm2_routed;  // second expert layer, routed experts
+  int gemm2_shared;  // second expert layer, shared expert
 };
 
 // Offsets of each workspace region (bytes), 256-byte aligned.
 struct WsLayout {
   size_t hdr, hist, base, tiles_simt, tiles_tc1, tiles_tc2, idx, w, counts, offsets, perm, inv,
-      logits, xp, hm, hs, yr, ys, stats, total;
+      logits, logits_part, xp, hm, hs, yr, ys, stats, total;
   int n_chunks;
   int max_tiles_simt, max_tiles_tc1, max_tiles_tc2;
+  Splits sp;
 };
 
 constexpr int kChunk = 2048;       // copies per dispatch chunk
 constexpr int kSimtRows = 64;      // rows per SIMT FFN tile
 constexpr int kTcRows = 256;       // max rows (MMA N) per tensor-core tile
+constexpr int kMaxSplits = 64;
 
+Splits choose_splits(const moe_layer_desc& d);
 WsLayout workspace_layout(const moe_layer_desc& d);
 void count_launch();   // bumps the process-wide kernel launch counter
 size_t dtype_size(int dtype);

@@ -15,12 +15,15 @@
 //                        __match_any_sync, so the order is ascending copy id.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
 __global__ void __launch_bounds__(256) chunk_histogram(const int32_t* __restrict__ idx, int TK,
                                                        int E, int32_t* __restrict__ hist,
                                                        uint32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int h[kMaxE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
   __syncthreads();
@@ -75,6 +78,7 @@ struct TileSpec {
   Tile* tc2;           // tensor-core tiles of GEMM2
   int m_tiles1_routed, m_tiles1_shared;   // output-column tiles (128 wide) of GEMM1
   int m_tiles2;                           // output-column tiles of GEMM2 (H / 128)
+  int splits2_routed, splits2_shared;     // reduction splits of GEMM2 tiles
 };
 
 // Number of balanced row tiles for a group of c rows and the rows per tile
@@ -110,38 +114,99 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
       t.r0 = r_base + i * kSimtRows;
       t.n = min(kSimtRows, g_rows - i * kSimtRows);
       t.m0 = 0;
+      t.ks = 0;
       ts.simt[first_simt + i] = t;
     }
   }
   // Tensor-core tiles: balanced row blocks (<= kTcRows rows, multiple of 16)
-  // times 128-wide output-column blocks.
+  // times 128-wide weight-row blocks. Order: the shared expert first, then
+  // the routed experts by descending row count (ties by index), so the
+  // longest work starts first; inside a group the weight-row blocks are
+  // outermost and the row blocks innermost, so the row blocks that share a
+  // 128-row weight slab run at the same time on neighbouring CTAs and read
+  // the slab from L2 instead of DRAM.
+  __shared__ int s_cnt[kMaxE];
+  __shared__ int s_pos1[kMaxE], s_pos2[kMaxE];
+  __shared__ int s_first1[kMaxE + 1], s_first2[kMaxE + 1], s_nt[kMaxE + 1], s_rper[kMaxE + 1],
+      s_rows[kMaxE + 1], s_rbase[kMaxE + 1];
   int nt_rows, rows_per;
   tc_row_split(g_rows, &nt_rows, &rows_per);
   const int mt1 = (e < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared;
+  int sh_nt, sh_rper;
+  tc_row_split(has_shared ? T : 0, &sh_nt, &sh_rper);
+  const int sh1 = sh_nt * ts.m_tiles1_shared, sh2 = sh_nt * ts.m_tiles2 * ts.splits2_shared;
+  if (e < E) s_cnt[e] = c;
+  __syncthreads();
+  int rank = 0;
+  if (e < E) {
+    for (int q = 0; q < E; ++q) {
+      const int cq = s_cnt[q];
+      rank += (cq > c) || (cq == c && q < e);
+    }
+    s_pos1[rank] = nt_rows * mt1;                  // tile counts in rank order
+    s_pos2[rank] = nt_rows * ts.m_tiles2 * ts.splits2_routed;
+  }
+  __syncthreads();
   int tot1, tot2;
-  const int first1 = block_exclusive_scan(nt_rows * mt1, sh, &tot1);
-  const int first2 = block_exclusive_scan(nt_rows * ts.m_tiles2, sh, &tot2);
+  const int p1 = block_exclusive_scan(e < E ? s_pos1[e] : 0, sh, &tot1);
+  const int p2 = block_exclusive_scan(e < E ? s_pos2[e] : 0, sh, &tot2);
+  if (e < E) {
+    s_pos1[e] = p1;
+    s_pos2[e] = p2;
+  }
+  __syncthreads();
+  if (e <= E) {
+    s_first1[e] = (e < E) ? sh1 + s_pos1[rank] : 0;
+    s_first2[e] = (e < E) ? sh2 + s_pos2[rank] : 0;
+    s_nt[e] = nt_rows;
+    s_rper[e] = rows_per;
+    s_rows[e] = g_rows;
+    s_rbase[e] = r_base;
+  }
+  __syncthreads();
   if (ts.tc1) {
-    int o1 = first1, o2 = first2;
-    for (int i = 0; i < nt_rows; ++i) {
-      Tile t;
-      t.g = e;
-      t.r0 = r_base + i * rows_per;
-      t.n = min(rows_per, g_rows - i * rows_per);
-      for (int m = 0; m < mt1; ++m) {
-        t.m0 = m * 128;
-        ts.tc1[o1++] = t;
-      }
-      for (int m = 0; m < ts.m_tiles2; ++m) {
-        t.m0 = m * 128;
-        ts.tc2[o2++] = t;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    for (int g = warp; g <= E; g += nwarps) {
+      const int nt = s_nt[g];
+      if (nt == 0) continue;
+      const int m1 = (g < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared;
+      const int sp2 = (g < E) ? ts.splits2_routed : ts.splits2_shared;
+      const int n1 = nt * m1, n2 = nt * ts.m_tiles2 * sp2;
+      for (int i = lane; i < n1 + n2; i += 32) {
+        const bool first = i < n1;
+        const int j = first ? i : i - n1;
+        const int sp = first ? 1 : sp2;
+        const int mt = first ? m1 : ts.m_tiles2;
+        // Order inside the group: when the group has more activation rows than
+        // weight rows the row blocks are outermost (the weight matrix stays in
+        // L2 while the rows stream once); otherwise the weight blocks are
+        // outermost (each weight slab streams once while its row blocks, on
+        // neighbouring CTAs, reuse it from L2). Splits vary fastest after that.
+        int r, q;
+        if (s_rows[g] > mt * 128) {
+          r = j / (mt * sp);
+          q = j - r * (mt * sp);
+        } else {
+          r = j % nt;
+          q = j / nt;
+        }
+        Tile t;
+        t.g = g;
+        t.r0 = s_rbase[g] + r * s_rper[g];
+        t.n = min(s_rper[g], s_rows[g] - r * s_rper[g]);
+        t.m0 = (q / sp) * 128;
+        t.ks = q % sp;
+        if (first)
+          ts.tc1[s_first1[g] + j] = t;
+        else
+          ts.tc2[s_first2[g] + j] = t;
       }
     }
   }
   if (threadIdx.x == 0) {
     hdr->n_tiles[0] = tot_simt;
-    hdr->n_tiles[1] = ts.tc1 ? tot1 : 0;
-    hdr->n_tiles[2] = ts.tc1 ? tot2 : 0;
+    hdr->n_tiles[1] = ts.tc1 ? tot1 + sh1 : 0;
+    hdr->n_tiles[2] = ts.tc1 ? tot2 + sh2 : 0;
   }
 }
 
@@ -151,20 +216,35 @@ __global__ void __launch_bounds__(1024) scan_and_tiles(const int32_t* __restrict
                                                        int32_t* __restrict__ offsets,
                                                        int32_t* __restrict__ base,
                                                        TileSpec ts, WsHeader* __restrict__ hdr) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int sh[96];
   const int e = threadIdx.x;   // one thread per expert slot (E <= 512 < 1024)
   int c = 0;
   if (e < E)
-    for (int k = 0; k < n_chunks; ++k) c += hist[(size_t)k * E + e];
+    for (int k0 = 0; k0 < n_chunks; k0 += 8) {   // 8 independent loads per round
+      int v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = (k0 + q < n_chunks) ? hist[(size_t)(k0 + q) * E + e] : 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) c += v[q];
+    }
   int total;
   const int off = block_exclusive_scan(e < E ? c : 0, sh, &total);
   if (e < E) {
     counts[e] = c;
     offsets[e] = off;
     int run = off;
-    for (int k = 0; k < n_chunks; ++k) {
-      base[(size_t)k * E + e] = run;
-      run += hist[(size_t)k * E + e];
+    for (int k0 = 0; k0 < n_chunks; k0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = (k0 + q < n_chunks) ? hist[(size_t)(k0 + q) * E + e] : 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (k0 + q < n_chunks) {
+          base[(size_t)(k0 + q) * E + e] = run;
+          run += v[q];
+        }
     }
   }
   if (e == E) offsets[E] = total;
@@ -176,6 +256,8 @@ __global__ void __launch_bounds__(1024) tiles_from_offsets(const int32_t* __rest
                                                            int E, int T, int has_shared,
                                                            TileSpec ts,
                                                            WsHeader* __restrict__ hdr) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int sh[96];
   const int e = threadIdx.x;
   int c = 0, off = 0;
@@ -192,6 +274,8 @@ __global__ void __launch_bounds__(256) chunk_scatter(const int32_t* __restrict__
                                                      int E, const int32_t* __restrict__ base,
                                                      int32_t* __restrict__ perm,
                                                      int32_t* __restrict__ inv) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int cnt[kScatterWarps][kMaxE];   // per-warp counts, then running ranks
   __shared__ int pre[kScatterWarps][kMaxE];   // exclusive prefix over warps
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -233,30 +317,115 @@ __global__ void __launch_bounds__(256) chunk_scatter(const int32_t* __restrict__
   }
 }
 
+// Dispatch of a small batch (T*K <= kChunk, every decode step) in one CTA:
+// the per-chunk histogram, the scan with the tile lists and the stable
+// scatter of the three kernels above, without their two launch gaps. Warp w
+// owns the consecutive copies [w * per_warp, (w + 1) * per_warp); counts per
+// (warp, expert) live in dynamic shared memory (32 * E ints, twice).
+constexpr int kSmallWarps = 32;
+
+__global__ void __launch_bounds__(1024) dispatch_small(const int32_t* __restrict__ idx, int TK,
+                                                       int E, int T, int has_shared,
+                                                       int32_t* __restrict__ counts,
+                                                       int32_t* __restrict__ offsets,
+                                                       int32_t* __restrict__ perm,
+                                                       int32_t* __restrict__ inv, TileSpec ts,
+                                                       WsHeader* __restrict__ hdr) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int dyn_smem[];
+  int* cnt = dyn_smem;                      // [kSmallWarps][E]
+  int* pre = dyn_smem + kSmallWarps * E;    // [kSmallWarps][E]
+  __shared__ int sh[96];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  const int per_warp = (TK + kSmallWarps - 1) / kSmallWarps;
+  const int w0 = min(TK, warp * per_warp), w1 = min(TK, w0 + per_warp);
+  bool bad = false;
+  for (int i = w0 + lane; i < w1; i += 32) {
+    const int e = idx[i];
+    if ((unsigned)e < (unsigned)E)
+      atomicAdd(&cnt[warp * E + e], 1);
+    else
+      bad = true;
+  }
+  if (bad) atomicOr(&hdr->status, kStatusBadIndex);
+  __syncthreads();
+  const int e = threadIdx.x;   // one thread per expert slot (E <= 512 < 1024)
+  int c = 0;
+  if (e < E)
+    for (int w = 0; w < kSmallWarps; ++w) c += cnt[w * E + e];
+  int total;
+  const int off = block_exclusive_scan(e < E ? c : 0, sh, &total);
+  if (e < E) {
+    counts[e] = c;
+    offsets[e] = off;
+    int run = off;
+    for (int w = 0; w < kSmallWarps; ++w) {
+      pre[w * E + e] = run;
+      run += cnt[w * E + e];
+      cnt[w * E + e] = 0;
+    }
+  }
+  if (e == E) offsets[E] = total;
+  emit_tiles(c, off, E, T, has_shared, ts, sh, hdr);
+  __syncthreads();
+  for (int i0 = w0; i0 < w1; i0 += 32) {
+    const int i = i0 + lane;
+    const bool live = i < w1;
+    const int ei = live ? idx[i] : -1;
+    const bool ok = live && (unsigned)ei < (unsigned)E;
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? ei : -1);
+    if (ok) {
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int row = pre[warp * E + ei] + cnt[warp * E + ei] + rank;
+      perm[row] = i;
+      inv[i] = row;
+    }
+    __syncwarp();
+    if (ok && (peers & ((1u << lane) - 1u)) == 0) cnt[warp * E + ei] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 // Gather of dispatched activation rows: xp[row] = x[perm[row] / K] (bf16,
 // 16-byte vectors), so the tensor-core GEMM reads contiguous rows.
 __global__ void __launch_bounds__(256) gather_rows(const uint4* __restrict__ x,
                                                    const int32_t* __restrict__ perm, int TK,
                                                    int K, int row_vecs, uint4* __restrict__ xp) {
-  const size_t total = (size_t)TK * row_vecs;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
-       i += (size_t)gridDim.x * blockDim.x) {
-    const size_t row = i / row_vecs;
-    const int v = (int)(i - row * row_vecs);
-    const int t = perm[row] / K;
-    xp[i] = x[(size_t)t * row_vecs + v];
+  pdl_wait();
+  pdl_trigger();
+  // one warp per row, 16-byte vectors, four in flight per lane
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < TK; row += warps) {
+    const uint4* src = x + (size_t)(perm[row] / K) * row_vecs;
+    uint4* dst = xp + (size_t)row * row_vecs;
+    for (int v0 = lane; v0 < row_vecs; v0 += 128) {
+      uint4 a[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (v0 + 32 * q < row_vecs) a[q] = src[v0 + 32 * q];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (v0 + 32 * q < row_vecs) dst[v0 + 32 * q] = a[q];
+    }
   }
 }
 
 static TileSpec make_tile_spec(const moe_layer_desc& d, const WsLayout& L, char* ws,
-                               bool tc_tiles) {
+                               bool tc_tiles, bool split) {
   TileSpec ts;
-  ts.simt = reinterpret_cast<Tile*>(ws + L.tiles_simt);
+  // CUDA-core tile lists only for layers that run the CUDA-core GEMM
+  ts.simt = tc_tiles ? nullptr : reinterpret_cast<Tile*>(ws + L.tiles_simt);
   ts.tc1 = tc_tiles ? reinterpret_cast<Tile*>(ws + L.tiles_tc1) : nullptr;
   ts.tc2 = tc_tiles ? reinterpret_cast<Tile*>(ws + L.tiles_tc2) : nullptr;
   ts.m_tiles1_routed = d.D / 128;
   ts.m_tiles1_shared = d.Ds / 128;
   ts.m_tiles2 = d.H / 128;
+  ts.splits2_routed = split ? L.sp.gemm2_routed : 1;
+  ts.splits2_shared = split ? L.sp.gemm2_shared : 1;
   return ts;
 }
 
@@ -268,21 +437,37 @@ cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
   int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
   const int n_chunks = L.n_chunks;
-  if (TK > 0) {
-    count_launch();
-    chunk_histogram<<<n_chunks, 256, 0, st>>>(idx, TK, d.E, hist, &hdr->status);
-  } else {
-    cudaMemsetAsync(hist, 0, sizeof(int32_t) * (size_t)n_chunks * d.E, st);
+  const TileSpec ts = make_tile_spec(d, L, ws, tc_tiles, /*split=*/true);
+  const int has_shared = d.Ds > 0 ? 1 : 0;
+  if (TK > 0 && TK <= kChunk) {
+    const size_t smem = sizeof(int) * 2 * kSmallWarps * (size_t)d.E;
+    static bool attr_set[64] = {false};   // per device: dynamic smem above 48 KB
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      e = cudaFuncSetAttribute(dispatch_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(sizeof(int) * 2 * kSmallWarps * kMaxE));
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    return launch_pdl(dispatch_small, dim3(1), dim3(1024), smem, st, idx, TK, d.E, d.T,
+                      has_shared, counts, offsets, perm, inv, ts, hdr);
   }
-  const TileSpec ts = make_tile_spec(d, L, ws, tc_tiles);
-  count_launch();
-  scan_and_tiles<<<1, 1024, 0, st>>>(hist, n_chunks, d.E, d.T, d.Ds > 0 ? 1 : 0, counts, offsets,
-                                     base, ts, hdr);
-  if (TK > 0) {
-    count_launch();
-    chunk_scatter<<<n_chunks, 256, 0, st>>>(idx, TK, d.E, base, perm, inv);
-  }
-  return cudaGetLastError();
+  cudaError_t e = cudaSuccess;
+  if (TK > 0)
+    e = launch_pdl(chunk_histogram, dim3(n_chunks), dim3(256), 0, st, idx, TK, d.E, hist,
+                   &hdr->status);
+  else
+    e = cudaMemsetAsync(hist, 0, sizeof(int32_t) * (size_t)n_chunks * d.E, st);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(scan_and_tiles, dim3(1), dim3(1024), 0, st, (const int32_t*)hist, n_chunks, d.E,
+                 d.T, has_shared, counts, offsets, base, ts, hdr);
+  if (e != cudaSuccess) return e;
+  if (TK > 0)
+    e = launch_pdl(chunk_scatter, dim3(n_chunks), dim3(256), 0, st, idx, TK, d.E,
+                   (const int32_t*)base, perm, inv);
+  return e;
 }
 
 // The same three dispatch kernels with caller-provided scratch: hist and base
@@ -312,11 +497,9 @@ cudaError_t launch_dispatch_scratch(const moe_layer_desc& d, int n_chunks, int32
 
 cudaError_t launch_tiles_from_offsets(const moe_layer_desc& d, const WsLayout& L, char* ws,
                                       const int32_t* offsets, bool tc_tiles, cudaStream_t st) {
-  const TileSpec ts = make_tile_spec(d, L, ws, tc_tiles);
-  count_launch();
-  tiles_from_offsets<<<1, 1024, 0, st>>>(offsets, d.E, d.T, d.Ds > 0 ? 1 : 0, ts,
-                                         reinterpret_cast<WsHeader*>(ws + L.hdr));
-  return cudaGetLastError();
+  const TileSpec ts = make_tile_spec(d, L, ws, tc_tiles, /*split=*/false);
+  return launch_pdl(tiles_from_offsets, dim3(1), dim3(1024), 0, st, offsets, d.E, d.T,
+                    d.Ds > 0 ? 1 : 0, ts, reinterpret_cast<WsHeader*>(ws + L.hdr));
 }
 
 cudaError_t launch_gather_rows(const moe_layer_desc& d, const void* x, const int32_t* perm,
@@ -324,11 +507,9 @@ cudaError_t launch_gather_rows(const moe_layer_desc& d, const void* x, const int
   const int TK = d.T * d.K;
   if (TK == 0) return cudaSuccess;
   const int row_vecs = d.H * 2 / 16;
-  const size_t total = (size_t)TK * row_vecs;
-  const int blocks = (int)std::min<size_t>((total + 255) / 256, (size_t)num_sms * 8);
-  count_launch();
-  gather_rows<<<blocks, 256, 0, st>>>((const uint4*)x, perm, TK, d.K, row_vecs, (uint4*)xp);
-  return cudaGetLastError();
+  const int blocks = (int)std::min<size_t>(((size_t)TK + 7) / 8, (size_t)num_sms * 8);   // 8 rows per block
+  return launch_pdl(gather_rows, dim3(blocks), dim3(256), 0, st, (const uint4*)x, perm, TK, d.K,
+                    row_vecs, (uint4*)xp);
 }
 
 }  // namespace moe

@@ -8,6 +8,7 @@
 // reads the GEMM1 rows directly. The shared expert is group E.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -20,6 +21,8 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt(const Tile* __restrict_
                                                          const int* __restrict__ n_tiles,
                                                          SimtProblem routed, SimtProblem shared,
                                                          int E) {
+  pdl_wait();
+  pdl_trigger();
   const int tile_id = blockIdx.x;
   if (tile_id >= *n_tiles) return;
   const Tile tl = tiles[tile_id];
@@ -100,9 +103,8 @@ static cudaError_t launch_simt_t(const SimtProblem& routed, const SimtProblem& s
                                  cudaStream_t st) {
   if (max_tiles <= 0) return cudaSuccess;
   dim3 grid(max_tiles, (max_n + kBN - 1) / kBN);
-  count_launch();
-  grouped_gemm_simt<TIn, TOut, kGelu><<<grid, 256, 0, st>>>(tiles, n_tiles, routed, shared, E);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_simt<TIn, TOut, kGelu>, grid, dim3(256), 0, st, tiles, n_tiles,
+                    routed, shared, E);
 }
 
 // First layer: output in the input dtype with GeLU; second layer: fp32

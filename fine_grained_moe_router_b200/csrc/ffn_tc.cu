@@ -9,14 +9,16 @@
 // handful of rows per expert still fills the 128-row MMA and the kernel
 // streams each touched weight slab once.
 //
-// Per CTA (persistent, one per SM, 192 threads):
-//   warp 4  TMA producer: weight slab [128 x 64] + activation rows [n x 64]
-//           per stage into 128-byte-swizzled shared memory, 4-stage ring
-//   warp 5  TMEM allocator and MMA issuer: tcgen05.mma kind::f16 (bf16 in,
+// Per CTA (persistent, one per SM, 320 threads):
+//   warp 8  TMA producer: weight slab [128 x 64] + activation rows [n x 64]
+//           per stage into 128-byte-swizzled shared memory; the ring has 4
+//           stages for 256-row tiles and up to 12 when the batch is small
+//   warp 9  TMEM allocator and MMA issuer: tcgen05.mma kind::f16 (bf16 in,
 //           fp32 accumulate), two 256-column TMEM accumulators so the
 //           epilogue of one tile overlaps the MMAs of the next
-//   warps 0-3  epilogue: tcgen05.ld of the accumulator (thread = weight row),
-//           exact GeLU for the first layer, bf16 stores into row-major output
+//   warps 0-7  epilogue: tcgen05.ld of the accumulator (thread = weight row,
+//           two warps per TMEM lane quarter splitting the columns), exact
+//           GeLU for the first layer, stores into row-major output
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // kStatusTimeout in the workspace, drains its in-flight copies and MMAs,
 // frees its TMEM and returns.
@@ -24,6 +26,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 namespace tc {
@@ -31,15 +34,17 @@ namespace tc {
 constexpr int kBM = 128;                        // weight rows per tile (MMA M)
 constexpr int kBK = 64;                         // reduction elements per stage (128 bytes)
 constexpr int kBoxRows = 32;                    // activation rows per TMA box
-constexpr int kStages = 4;
+constexpr int kBoxBytes = kBoxRows * kBK * 2;   // 4 KB
 constexpr int kABytes = kBM * kBK * 2;          // 16 KB
-constexpr int kBBytes = kTcRows * kBK * 2;      // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kMaxStages = 12;
+constexpr int kStageArea = 192 * 1024;          // shared memory of the operand ring
 constexpr int kAccCols = 256;                   // fp32 columns per accumulator
 constexpr int kTmemCols = 2 * kAccCols;
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
-constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256;
+constexpr int kEpiWarps = 8;                    // two per TMEM lane quarter
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
+constexpr int kThreads = (kEpiWarps + 2) * 32;
+constexpr size_t kSmemBytes = 1024 /*barriers*/ + 1024 /*alignment*/ + kStageArea;
 constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s bound on any wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -154,22 +159,45 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-struct Side {        // routed experts (0) or the shared expert (1)
-  void* out;         // output rows, row stride `ld` elements
+struct Side {          // routed experts (0) or the shared expert (1)
+  void* out;           // output rows, row stride `ld` elements
+  long long split_stride;   // elements between the partial outputs of two splits
   int ld;
-  int kb;            // reduction blocks of kBK
-  int m_rows;        // weight rows per group (row stride of groups in the A map)
-  int out_f32;       // 1: fp32 output, 0: bf16 output
+  int kb;              // reduction blocks of kBK
+  int kb_per;          // reduction blocks per split
+  int m_rows;          // weight rows per group (row stride of groups in the A map)
+  int m_valid;         // output columns below this bound are stored
+  int out_f32;         // 1: fp32 output, 0: bf16 output
+  int a_rows;          // rows of the weight box (kBM, or fewer for a short gate matrix)
 };
 
 struct Args {
   Side side[2];
-  const Tile* tiles;
-  const int* n_tiles;
+  const Tile* tiles;   // device tile list; null: dense tiling (below)
+  const int* n_tiles;  // device tile count of the list
+  int dense_tiles;     // dense tiling: row tiles x weight-row tiles x splits
+  int dense_rows, dense_m_tiles, dense_splits;
+  int nbox_max;        // activation boxes per stage (rows per tile <= 32 * nbox_max)
+  int stage_bytes;     // kABytes + nbox_max * kBoxBytes
+  int n_stages;        // stages in the ring (<= kMaxStages)
   uint32_t* status;
   int E;
   int gelu;
 };
+
+// Tile t of the launch: from the list, or (dense tiling, used by the gate
+// GEMM) split fastest, then weight-row block, then row block.
+__device__ __forceinline__ Tile tile_at(const Args& a, int t) {
+  if (a.tiles) return a.tiles[t];
+  Tile tl;
+  tl.ks = t % a.dense_splits;
+  const int q = t / a.dense_splits;
+  tl.m0 = (q % a.dense_m_tiles) * kBM;
+  tl.r0 = (q / a.dense_m_tiles) * kTcRows;
+  tl.n = min(kTcRows, a.dense_rows - tl.r0);
+  tl.g = 0;
+  return tl;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA0,
@@ -177,20 +205,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB1, const Args args) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
+  uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * kStageBytes);
-  uint64_t* full = bars;                   // [kStages] TMA landed
-  uint64_t* empty = bars + kStages;        // [kStages] MMAs done reading
-  uint64_t* tfull = bars + 2 * kStages;    // [2] accumulator ready
-  uint64_t* tempty = bars + 2 * kStages + 2;   // [2] accumulator drained
-  uint64_t* drain = bars + 2 * kStages + 4;    // [1] all MMAs retired
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base);     // first 1 KB: control
+  uint64_t* full = bars;                                  // [kMaxStages] TMA landed
+  uint64_t* empty = bars + kMaxStages;                    // [kMaxStages] MMAs done reading
+  uint64_t* tfull = bars + 2 * kMaxStages;                // [2] accumulator ready
+  uint64_t* tempty = bars + 2 * kMaxStages + 2;           // [2] accumulator drained
+  uint64_t* drain = bars + 2 * kMaxStages + 4;            // [1] all MMAs retired
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMaxStages + 5);
   volatile uint32_t* abort_flag = tmem_slot + 1;
+  uint8_t* ring = base + 1024;                            // stage s at s * stage_bytes
+  const int n_stages = args.n_stages;
+  const int stage_bytes = args.stage_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < n_stages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
@@ -203,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(kTmemCols));
@@ -213,78 +244,91 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int n_tiles = *args.n_tiles;
+  // the prologue above overlaps the previous kernel; its outputs are read below
+  pdl_wait();
+  pdl_trigger();
+  const int n_tiles = args.tiles ? *args.n_tiles : args.dense_tiles;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued_parity[kStages];
-      bool issued[kStages];
-      for (int s = 0; s < kStages; ++s) issued[s] = false, issued_parity[s] = 0;
+      uint32_t issued_parity[kMaxStages];
+      bool issued[kMaxStages];
+      for (int s = 0; s < kMaxStages; ++s) issued[s] = false, issued_parity[s] = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-        const Tile tl = args.tiles[t];
+        const Tile tl = tile_at(args, t);
         const int sd = (tl.g < args.E) ? 0 : 1;
         const Side& S = args.side[sd];
         const CUtensorMap* ma = sd ? &tmA1 : &tmA0;
         const CUtensorMap* mb = sd ? &tmB1 : &tmB0;
         const int arow = (sd ? 0 : tl.g * S.m_rows) + tl.m0;
         const int nmma = (tl.n + 15) & ~15;
-        const int nbox = (nmma + kBoxRows - 1) / kBoxRows;
-        const uint32_t bytes = kABytes + nbox * kBoxRows * kBK * 2;
-        for (int kb = 0; kb < S.kb; ++kb) {
+        int nbox = (nmma + kBoxRows - 1) / kBoxRows;
+        if (nbox > args.nbox_max) {   // never by construction; keeps the ring in bounds
+          atomicOr(args.status, kStatusBadIndex);
+          nbox = args.nbox_max;
+        }
+        // weight rows actually loaded: 128, or fewer for a gate matrix with
+        // E < 128 rows (the other rows of the smem tile only feed outputs
+        // that are never stored)
+        const uint32_t bytes = (uint32_t)S.a_rows * kBK * 2 + (uint32_t)nbox * kBoxBytes;
+        const int kb0 = tl.ks * S.kb_per, kb1 = min(S.kb, kb0 + S.kb_per);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
           }
           const uint32_t fb = smem_u32(&full[stage]);
           mbar_expect_tx(fb, bytes);
-          const uint32_t sa = smem_u32(smem + (size_t)stage * kStageBytes);
+          const uint32_t sa = smem_u32(ring + (size_t)stage * stage_bytes);
           const uint32_t sb = sa + kABytes;
           tma_load_2d(sa, ma, kb * kBK, arow, fb);
           for (int i = 0; i < nbox; ++i)
-            tma_load_2d(sb + i * kBoxRows * kBK * 2, mb, kb * kBK, tl.r0 + i * kBoxRows, fb);
+            tma_load_2d(sb + i * kBoxBytes, mb, kb * kBK, tl.r0 + i * kBoxRows, fb);
           issued[stage] = true;
           issued_parity[stage] = phase;
-          if (++stage == kStages) {
+          if (++stage == n_stages) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
       // every copy this thread started has landed before the CTA tears down
-      for (int s = 0; s < kStages; ++s)
+      for (int s = 0; s < n_stages; ++s)
         if (issued[s]) wait_bounded(smem_u32(&full[s]), issued_parity[s], nullptr, args.status);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-        const Tile tl = args.tiles[t];
+        const Tile tl = tile_at(args, t);
         const Side& S = args.side[(tl.g < args.E) ? 0 : 1];
-        const uint32_t idesc = idesc_bf16((tl.n + 15) & ~15);
+        const int nmma = min((tl.n + 15) & ~15, args.nbox_max * kBoxRows);
+        const uint32_t idesc = idesc_bf16(nmma);
+        const int kb0 = tl.ks * S.kb_per, kb1 = min(S.kb, kb0 + S.kb_per);
         if (!wait_bounded(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
-        for (int kb = 0; kb < S.kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_bounded(smem_u32(&full[stage]), phase, abort_flag, args.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + (size_t)stage * kStageBytes);
+          const uint32_t sa = smem_u32(ring + (size_t)stage * stage_bytes);
           const uint64_t adesc = sw128_desc(sa);
           const uint64_t bdesc = sw128_desc(sa + kABytes);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)   // 16 elements = 32 bytes per MMA
-            mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+            mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
           mma_commit(smem_u32(&empty[stage]));
-          if (++stage == kStages) {
+          if (++stage == n_stages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -302,11 +346,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // --------------------------------------------------------- epilogue
+    // warp w reads TMEM lanes 32*(w%4) .. +31 (thread = weight row of the
+    // tile) and the 32-column chunks (w/4), (w/4)+2, ... of the accumulator
+    // (column = activation row of the tile).
     int acc = 0;
     uint32_t acc_phase = 0;
-    const int row = warp * 32 + lane;   // weight row of this thread within the tile
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-      const Tile tl = args.tiles[t];
+      const Tile tl = tile_at(args, t);
       const int sd = (tl.g < args.E) ? 0 : 1;
       const Side& S = args.side[sd];
       int ok = 1;
@@ -316,22 +364,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t taddr =
-          tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * kAccCols);
-      const size_t col = (size_t)tl.m0 + row;
-      for (int c0 = 0; c0 < tl.n; c0 += 32) {
+          tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kAccCols);
+      const int col = tl.m0 + row;
+      const bool store = col < S.m_valid;
+      const size_t part = (size_t)tl.ks * (size_t)S.split_stride;
+      const int n = min(tl.n, args.nbox_max * kBoxRows);
+      for (int c0 = half * 32; c0 < n; c0 += 64) {
         uint32_t r[32];
+        __syncwarp();
         tmem_ld32(taddr + (uint32_t)c0, r);
+        if (store) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int j = c0 + q;
-          if (j < tl.n) {
-            float v = __uint_as_float(r[q]);
-            if (args.gelu) v = gelu_erf(v);
-            const size_t o = (size_t)(tl.r0 + j) * S.ld + col;
-            if (S.out_f32)
-              static_cast<float*>(S.out)[o] = v;
-            else
-              static_cast<__nv_bfloat16*>(S.out)[o] = __float2bfloat16_rn(v);
+          for (int q = 0; q < 32; ++q) {
+            const int j = c0 + q;
+            if (j < n) {
+              float v = __uint_as_float(r[q]);
+              if (args.gelu) v = gelu_erf(v);
+              const size_t o = part + (size_t)(tl.r0 + j) * S.ld + col;
+              if (S.out_f32)
+                static_cast<float*>(S.out)[o] = v;
+              else
+                static_cast<__nv_bfloat16*>(S.out)[o] = __float2bfloat16_rn(v);
+            }
           }
         }
       }
@@ -346,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(kTmemCols));
@@ -391,7 +445,8 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
 
 cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& shared, int E,
                                    bool gelu, const Tile* tiles, const int* n_tiles,
-                                   uint32_t* status, int num_sms, cudaStream_t st) {
+                                   const DenseTiling* dense, uint32_t* status, int num_sms,
+                                   cudaStream_t st) {
   using namespace tc;
   static bool attr_set[64] = {false};   // per device
   int dev = 0;
@@ -403,25 +458,57 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
+  // A weight matrix shorter than one tile (a gate matrix with E < 128) is
+  // loaded with a box of its own rows rounded up to a swizzle atom (8 rows).
+  auto a_rows_of = [](const TcProblem& p) {
+    return p.w_rows >= (uint64_t)kBM ? kBM : (int)((p.w_rows + 7) & ~7ull);
+  };
   CUtensorMap a0, b0, a1, b1;
-  if (!make_map(&a0, routed.w, routed.w_rows, routed.kd, kBM) ||
+  if (!make_map(&a0, routed.w, routed.w_rows, routed.kd, a_rows_of(routed)) ||
       !make_map(&b0, routed.act, routed.act_rows, routed.kd, kBoxRows))
     return cudaErrorInvalidValue;
   const TcProblem& sh = shared.w ? shared : routed;   // unused maps still need valid encodings
-  if (!make_map(&a1, sh.w, sh.w_rows, sh.kd, kBM) ||
+  if (!make_map(&a1, sh.w, sh.w_rows, sh.kd, a_rows_of(sh)) ||
       !make_map(&b1, sh.act, sh.act_rows, sh.kd, kBoxRows))
     return cudaErrorInvalidValue;
+  auto side = [&](const TcProblem& p) {
+    Side s;
+    s.a_rows = a_rows_of(p);
+    s.out = p.out;
+    s.split_stride = p.split_stride;
+    s.ld = p.ld;
+    s.kb = p.kd / kBK;
+    const int splits = p.splits > 0 ? p.splits : 1;
+    s.kb_per = (s.kb + splits - 1) / splits;
+    s.m_rows = p.m_rows;
+    s.m_valid = p.m_valid > 0 ? p.m_valid : p.m_rows;
+    s.out_f32 = p.out_f32 ? 1 : 0;
+    return s;
+  };
   Args args;
-  args.side[0] = Side{routed.out, routed.ld, routed.kd / kBK, routed.m_rows, routed.out_f32};
-  args.side[1] = Side{sh.out, sh.ld, sh.kd / kBK, sh.m_rows, sh.out_f32};
-  args.tiles = tiles;
+  args.side[0] = side(routed);
+  args.side[1] = side(sh);
+  args.tiles = dense ? nullptr : tiles;
   args.n_tiles = n_tiles;
+  args.dense_tiles = dense ? dense->tiles : 0;
+  args.dense_rows = dense ? dense->rows : 0;
+  args.dense_m_tiles = dense ? dense->m_tiles : 1;
+  args.dense_splits = dense ? (routed.splits > 0 ? routed.splits : 1) : 1;
+  // Ring shape: no tile has more rows than its activation matrix, so small
+  // batches get small activation boxes per stage and a deeper ring (more
+  // weight bytes in flight per SM).
+  uint64_t rows = routed.act_rows;
+  if (shared.w) rows = std::max<uint64_t>(rows, shared.act_rows);
+  const int max_n = (int)std::min<uint64_t>(kTcRows, (rows + 15) & ~15ull);
+  args.nbox_max = (max_n + kBoxRows - 1) / kBoxRows;
+  args.stage_bytes = kABytes + args.nbox_max * kBoxBytes;
+  args.n_stages = std::min(kMaxStages, kStageArea / args.stage_bytes);
   args.status = status;
   args.E = E;
   args.gelu = gelu ? 1 : 0;
-  count_launch();
-  grouped_gemm_tc<<<num_sms, kThreads, kSmemBytes, st>>>(a0, b0, a1, b1, args);
-  return cudaGetLastError();
+  const int grid = dense ? std::min(num_sms, std::max(1, dense->tiles)) : num_sms;
+  return launch_pdl(grouped_gemm_tc, dim3(grid), dim3(kThreads), kSmemBytes, st, a0, b0, a1, b1,
+                    args);
 }
 
 }  // namespace moe

@@ -30,16 +30,32 @@ struct TcProblem {
   void* out;               // [*, ld], bf16 (first layer) or fp32 (out_f32)
   int ld;
   bool out_f32;
+  int splits;              // reduction splits (0 or 1: none); split s writes out + s * split_stride
+  long long split_stride;
+  int m_valid;             // output columns stored (0: all m_rows)
+};
+
+// Tiling without a device tile list (gate GEMM): `rows` activation rows in
+// blocks of kTcRows, `m_tiles` weight-row blocks, routed.splits splits.
+struct DenseTiling {
+  int tiles, rows, m_tiles;
 };
 
 cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& shared, int E,
                                    bool gelu, const Tile* tiles, const int* n_tiles,
-                                   uint32_t* status, int num_sms, cudaStream_t st);
+                                   const DenseTiling* dense, uint32_t* status, int num_sms,
+                                   cudaStream_t st);
 
 cudaError_t launch_gate_logits(const moe_layer_desc& d, const void* x, const void* wr,
                                float* logits, cudaStream_t st);
-cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, const float* bias,
-                               int32_t* idx, float* w, cudaStream_t st);
+cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, int n_parts,
+                               size_t part_stride, const float* bias, int32_t* idx, float* w,
+                               float* logits_out, cudaStream_t st);
+// Gate logits on the tensor cores (bf16 layers): `parts` receives
+// L.sp.router partial sums [T, E] fp32, part stride T * E.
+cudaError_t launch_gate_logits_tc(const moe_layer_desc& d, const WsLayout& L, char* ws,
+                                  const void* x, const void* wr, float* parts, int num_sms,
+                                  cudaStream_t st);
 cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws,
                             const int32_t* idx, int32_t* counts, int32_t* offsets,
                             int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st);
@@ -55,8 +71,11 @@ cudaError_t launch_grouped_gemm_simt(int dtype, bool gelu, const SimtProblem& ro
                                      const SimtProblem& shared, int E, const Tile* tiles,
                                      const int* n_tiles, int max_tiles, int max_n,
                                      cudaStream_t st);
+// y_rows / y_shared may hold several partial sums (reduction splits of the
+// second expert GEMM), T*K*H and T*H elements apart.
 cudaError_t launch_combine(const moe_layer_desc& d, const void* y_rows, const float* w,
-                           const int32_t* inv, const void* y_shared, void* y, cudaStream_t st);
+                           const int32_t* inv, const void* y_shared, void* y, cudaStream_t st,
+                           int rows_parts = 1, int shared_parts = 1);
 cudaError_t launch_expert_stats(const moe_layer_desc& d, const int32_t* counts, uint8_t* mask,
                                 moe_stats* out_dev, cudaStream_t st);
 

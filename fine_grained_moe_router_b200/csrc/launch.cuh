@@ -1,0 +1,39 @@
+// Kernel launches with programmatic dependent launch (PDL).
+//
+// Each kernel of the layer forward is launched with programmatic stream
+// serialization allowed, so the GPU can start scheduling it while the
+// previous kernel drains. Every such kernel calls pdl_wait() before its
+// first global-memory access: it returns once the preceding grid has
+// completed and its writes are visible, so data dependencies are exactly as
+// with ordinary stream order. pdl_trigger() lets the next kernel launch.
+#pragma once
+
+#include <utility>
+
+#include "common.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+}  // namespace moe

@@ -9,6 +9,7 @@
 // chosen set is the same, and ties stay exact ties (lower expert index wins).
 #include "common.cuh"
 #include "kernels.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -47,6 +48,8 @@ __global__ void __launch_bounds__(256) gate_logits_simt(const TIn* __restrict__ 
                                                         const TIn* __restrict__ wr,
                                                         float* __restrict__ logits, int T,
                                                         int H, int E) {
+  pdl_wait();
+  pdl_trigger();
   using V = Vec<TIn>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * kGateExp + warp;
@@ -94,19 +97,33 @@ __device__ __forceinline__ bool better(float sa, int ea, float sb, int eb) {
   return sa > sb || (sa == sb && ea < eb);
 }
 
+// lrow: the token's logits, given as n_parts partial sums part_stride apart
+// (reduction splits of the gate GEMM), added in split order; the total is
+// written to logits_out when it is non-null.
 template <int NJ>
-__device__ __forceinline__ void select_row(const float* __restrict__ lrow,
-                                           const float* __restrict__ bias, int E, int K,
-                                           int32_t* __restrict__ idx_out,
-                                           float* __restrict__ w_out) {
+__device__ __forceinline__ void select_row(const float* __restrict__ lrow, int n_parts,
+                                           size_t part_stride, const float* __restrict__ bias,
+                                           int E, int K, int32_t* __restrict__ idx_out,
+                                           float* __restrict__ w_out,
+                                           float* __restrict__ logits_out) {
   const int lane = threadIdx.x & 31;
   float s[NJ];
 #pragma unroll
   for (int j = 0; j < NJ; ++j) {
     const int e = lane + 32 * j;
     if (e < E) {
+      float l = lrow[e];
+      for (int p0 = 1; p0 < n_parts; p0 += 8) {   // 8 independent loads, then in-order adds
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = (p0 + q < n_parts) ? lrow[(p0 + q) * part_stride + e] : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (p0 + q < n_parts) l = __fadd_rn(l, v[q]);
+      }
+      if (logits_out) logits_out[e] = l;
       const float b = bias ? bias[e] : 0.f;
-      s[j] = __fadd_rn(lrow[e], b);
+      s[j] = __fadd_rn(l, b);
     } else {
       s[j] = -INFINITY;
     }
@@ -153,13 +170,18 @@ __device__ __forceinline__ void select_row(const float* __restrict__ lrow,
 
 template <int NJ>
 __global__ void __launch_bounds__(256) topk_select_kernel(const float* __restrict__ logits,
+                                                          int n_parts, size_t part_stride,
                                                           const float* __restrict__ bias, int T,
                                                           int E, int K,
                                                           int32_t* __restrict__ idx,
-                                                          float* __restrict__ w) {
+                                                          float* __restrict__ w,
+                                                          float* __restrict__ logits_out) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
-  select_row<NJ>(logits + (size_t)t * E, bias, E, K, idx + (size_t)t * K, w + (size_t)t * K);
+  select_row<NJ>(logits + (size_t)t * E, n_parts, part_stride, bias, E, K, idx + (size_t)t * K,
+                 w + (size_t)t * K, logits_out ? logits_out + (size_t)t * E : nullptr);
 }
 
 // ---------------------------------------------------------------------------
@@ -169,23 +191,54 @@ cudaError_t launch_gate_logits(const moe_layer_desc& d, const void* x, const voi
                                float* logits, cudaStream_t st) {
   if (d.T == 0) return cudaSuccess;
   dim3 grid((d.E + kGateExp - 1) / kGateExp, (d.T + kGateTok - 1) / kGateTok);
-  count_launch();
   if (d.dtype == MOE_BF16)
-    gate_logits_simt<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)wr, logits, d.T, d.H, d.E);
-  else
-    gate_logits_simt<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)wr, logits,
-                                                  d.T, d.H, d.E);
-  return cudaGetLastError();
+    return launch_pdl(gate_logits_simt<__nv_bfloat16>, grid, dim3(256), 0, st,
+                      (const __nv_bfloat16*)x, (const __nv_bfloat16*)wr, logits, d.T, d.H, d.E);
+  return launch_pdl(gate_logits_simt<float>, grid, dim3(256), 0, st, (const float*)x,
+                    (const float*)wr, logits, d.T, d.H, d.E);
 }
 
-cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, const float* bias,
-                               int32_t* idx, float* w, cudaStream_t st) {
+// Gate GEMM of bf16 layers on the tensor cores: W_r is operand A (expert
+// rows, one or more 128-row blocks; rows past E are zero-filled by TMA and
+// their outputs are not stored), x is operand B (token rows). With several
+// reduction splits each split writes its own fp32 partial [T, E]; the
+// selection kernel adds them in split order.
+cudaError_t launch_gate_logits_tc(const moe_layer_desc& d, const WsLayout& L, char* ws,
+                                  const void* x, const void* wr, float* parts, int num_sms,
+                                  cudaStream_t st) {
+  if (d.T == 0) return cudaSuccess;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
+  TcProblem p{};
+  p.act = x;
+  p.act_rows = (uint64_t)d.T;
+  p.w = wr;
+  p.w_rows = (uint64_t)d.E;
+  p.m_rows = d.E;
+  p.kd = d.H;
+  p.out = parts;
+  p.ld = d.E;
+  p.out_f32 = true;
+  p.splits = L.sp.router;
+  p.split_stride = (long long)d.T * d.E;
+  p.m_valid = d.E;
+  DenseTiling dense;
+  dense.rows = d.T;
+  dense.m_tiles = (d.E + 127) / 128;
+  dense.tiles = ((d.T + kTcRows - 1) / kTcRows) * dense.m_tiles * L.sp.router;
+  return launch_grouped_gemm_tc(p, TcProblem{}, d.E, false, nullptr, nullptr, &dense,
+                                &hdr->status, num_sms, st);
+}
+
+cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, int n_parts,
+                               size_t part_stride, const float* bias, int32_t* idx, float* w,
+                               float* logits_out, cudaStream_t st) {
   if (d.T == 0) return cudaSuccess;
   const int nj = (d.E + 31) / 32;
   dim3 grid((d.T + 7) / 8);
-#define MOE_TOPK_CASE(NJ) \
-  case NJ: count_launch(); topk_select_kernel<NJ><<<grid, 256, 0, st>>>(logits, bias, d.T, d.E, d.K, idx, w); break;
+#define MOE_TOPK_CASE(NJ)                                                                    \
+  case NJ:                                                                                   \
+    return launch_pdl(topk_select_kernel<NJ>, grid, dim3(256), 0, st, logits, n_parts,       \
+                      part_stride, bias, d.T, d.E, d.K, idx, w, logits_out);
   switch (nj) {
     MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4)
     MOE_TOPK_CASE(5) MOE_TOPK_CASE(6) MOE_TOPK_CASE(7) MOE_TOPK_CASE(8)

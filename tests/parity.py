@@ -81,7 +81,10 @@ def compare_routing(wl, gpu_logits, gpu_idx, gpu_w, ref_logits64, bias):
     uniq = unique_selection_mask(s64, K, tol)
     ref_idx, ref_w, _ = oracle.select_topk(ref_logits64, bias, K)
     assert (gpu_idx[uniq] == ref_idx[uniq]).all(), "selection differs on a token with a unique answer"
-    assert np.max(np.abs(gpu_w[uniq] - ref_w[uniq]), initial=0.0) <= W_TOL
+    # w_k = softmax of the chosen scores: dw_k/ds_j = w_k (delta_kj - w_j), so a
+    # score error e moves each weight by at most 2 e (plus fp32 rounding).
+    w_tol = W_TOL + 2.0 * tol
+    assert np.max(np.abs(gpu_w[uniq] - ref_w[uniq]), initial=0.0) <= w_tol
     if (~uniq).any():
         check_selection_valid(gpu_idx[~uniq], s64[~uniq], tol)
     np.testing.assert_allclose(gpu_w.sum(axis=1), 1.0, atol=1e-6)
