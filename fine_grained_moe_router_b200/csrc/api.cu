@@ -32,20 +32,24 @@ static int split_count(long long tiles, int kb, int want_tiles, int min_kb) {
 }
 
 Splits choose_splits(const moe_layer_desc& d) {
-  Splits s{1, 1, 1};
+  Splits s{1, 1, 1, 0};
   if (d.dtype != MOE_BF16 || d.T == 0) return s;
-  constexpr int kTargetTiles = 296;   // two per SM
   const long long T = d.T, TK = (long long)d.T * d.K;
+  // CTA pairs (256 weight rows per tile) when the touched experts average
+  // at least 64 rows each: then the tiles are wide enough in N for the
+  // halved per-SM operand traffic to matter.
+  const long long touched = std::min<long long>(d.E, TK);
+  s.pair = (d.D % 256 == 0 && d.H % 256 == 0 && d.Ds % 256 == 0 && TK >= 64 * touched) ? 1 : 0;
+  const int kTargetTiles = s.pair ? 148 : 296;   // two per SM or per pair
   const long long row_tiles = (T + kTcRows - 1) / kTcRows;
-  s.router = std::min(16, split_count(row_tiles * ((d.E + 127) / 128), d.H / 64,
-                                      kTargetTiles / 2, 2));
+  s.router = std::min(16, split_count(row_tiles * ((d.E + 127) / 128), d.H / 64, 148, 2));
   {  // no empty split after the cap
     const int kb = d.H / 64, per = (kb + s.router - 1) / s.router;
     s.router = (kb + per - 1) / per;
   }
   // GEMM2: each touched expert has at least one row tile; a decode step
   // touches min(E, T*K) experts.
-  const int mt2 = d.H / 128;
+  const int mt2 = d.H / (s.pair ? 256 : 128);
   const long long r_tiles = std::max(std::min<long long>(d.E, TK), (TK + kTcRows - 1) / kTcRows) * mt2;
   const long long s_tiles = d.Ds ? row_tiles * mt2 : 0;
   if (r_tiles + s_tiles < kTargetTiles) {
@@ -194,13 +198,17 @@ static moe_status run_grouped_ffn(const moe_layer_desc& d, const WsLayout& L, ch
       s2 = problem(hs, (uint64_t)d.T, ws2, (uint64_t)d.H, d.H, d.Ds, y_shared, d.H, true, sp_s,
                    (long long)d.T * d.H);
     }
+    // the tile lists of a split (layer-forward) dispatch follow L.sp.pair
+    const bool pair = split && L.sp.pair;
     MOE_CUDA_TRY(launch_grouped_gemm_tc(r1, s1, d.E, true,
                                         reinterpret_cast<const Tile*>(ws + L.tiles_tc1),
-                                        &hdr->n_tiles[1], nullptr, &hdr->status, num_sms(), st));
+                                        &hdr->n_tiles[1], nullptr, pair, &hdr->status, num_sms(),
+                                        st));
     if (ev_after_gemm1) MOE_CUDA_TRY(cudaEventRecord(*ev_after_gemm1, st));
     MOE_CUDA_TRY(launch_grouped_gemm_tc(r2, s2, d.E, false,
                                         reinterpret_cast<const Tile*>(ws + L.tiles_tc2),
-                                        &hdr->n_tiles[2], nullptr, &hdr->status, num_sms(), st));
+                                        &hdr->n_tiles[2], nullptr, pair, &hdr->status, num_sms(),
+                                        st));
     return MOE_OK;
   }
   SimtProblem r1{x, perm, d.K, w1, (size_t)d.D * d.H, hm, d.H, d.D};

@@ -62,6 +62,7 @@ struct Splits {
   int router;        // gate GEMM
   int gemm2_routed;  // second expert layer, routed experts
   int gemm2_shared;  // second expert layer, shared expert
+  int pair;          // 1: expert GEMMs on CTA pairs (256 weight rows per tile)
 };
 
 // Offsets of each workspace region (bytes), 256-byte aligned.

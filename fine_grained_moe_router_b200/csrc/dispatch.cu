@@ -79,6 +79,7 @@ struct TileSpec {
   int m_tiles1_routed, m_tiles1_shared;   // output-column tiles (128 wide) of GEMM1
   int m_tiles2;                           // output-column tiles of GEMM2 (H / 128)
   int splits2_routed, splits2_shared;     // reduction splits of GEMM2 tiles
+  int mtile;                              // weight rows per tile: 128, or 256 on CTA pairs
 };
 
 // Number of balanced row tiles for a group of c rows and the rows per tile
@@ -183,7 +184,7 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
         // outermost (each weight slab streams once while its row blocks, on
         // neighbouring CTAs, reuse it from L2). Splits vary fastest after that.
         int r, q;
-        if (s_rows[g] > mt * 128) {
+        if (s_rows[g] > mt * ts.mtile) {
           r = j / (mt * sp);
           q = j - r * (mt * sp);
         } else {
@@ -194,7 +195,7 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
         t.g = g;
         t.r0 = s_rbase[g] + r * s_rper[g];
         t.n = min(s_rper[g], s_rows[g] - r * s_rper[g]);
-        t.m0 = (q / sp) * 128;
+        t.m0 = (q / sp) * ts.mtile;
         t.ks = q % sp;
         if (first)
           ts.tc1[s_first1[g] + j] = t;
@@ -421,9 +422,10 @@ static TileSpec make_tile_spec(const moe_layer_desc& d, const WsLayout& L, char*
   ts.simt = tc_tiles ? nullptr : reinterpret_cast<Tile*>(ws + L.tiles_simt);
   ts.tc1 = tc_tiles ? reinterpret_cast<Tile*>(ws + L.tiles_tc1) : nullptr;
   ts.tc2 = tc_tiles ? reinterpret_cast<Tile*>(ws + L.tiles_tc2) : nullptr;
-  ts.m_tiles1_routed = d.D / 128;
-  ts.m_tiles1_shared = d.Ds / 128;
-  ts.m_tiles2 = d.H / 128;
+  ts.mtile = (split && L.sp.pair) ? 256 : 128;
+  ts.m_tiles1_routed = d.D / ts.mtile;
+  ts.m_tiles1_shared = d.Ds / ts.mtile;
+  ts.m_tiles2 = d.H / ts.mtile;
   ts.splits2_routed = split ? L.sp.gemm2_routed : 1;
   ts.splits2_shared = split ? L.sp.gemm2_shared : 1;
   return ts;

@@ -119,10 +119,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor of kind::f16: bf16 A and B (both K-major), fp32
-// accumulator, M = 128, N = n (multiple of 16, <= 256).
-__device__ __forceinline__ uint32_t idesc_bf16(int n) {
+// accumulator, M = m (128, or 256 for a CTA pair), N = n (multiple of 16,
+// <= 256).
+__device__ __forceinline__ uint32_t idesc_bf16(int n, int m) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(kBM >> 4) << 24);
+         ((uint32_t)(m >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
@@ -143,6 +144,57 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// ---- CTA-pair (cta_group::2) forms: two SMs of a cluster share one MMA
+// of M = 256; each holds half of the weight rows and half of the
+// activation rows of every stage, and its own half of the accumulator.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (here always the leader's).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x,
+                                                 int y, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t a, uint64_t b,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+// Arrive on the barrier at this offset in both CTAs of the pair once every
+// MMA issued so far has completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -199,6 +251,12 @@ __device__ __forceinline__ Tile tile_at(const Args& a, int t) {
   return tl;
 }
 
+// kPair = false: one CTA per tile of 128 weight rows (MMA M = 128).
+// kPair = true: a cluster of two CTAs per tile of 256 weight rows (one MMA of
+// M = 256 issued by the even CTA); each CTA loads its 128 weight rows and half
+// of the tile's activation rows per stage, so an SM streams a third less
+// operand data per MMA cycle than with single-CTA tiles of the same N.
+template <bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmB0,
@@ -218,6 +276,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ring = base + 1024;                            // stage s at s * stage_bytes
   const int n_stages = args.n_stages;
   const int stage_bytes = args.stage_bytes;
+  const uint32_t rank = kPair ? cluster_rank() : 0u;     // 0: the CTA that issues the MMAs
+  const bool leader = rank == 0;
+  const int unit = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int n_units = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  constexpr int kTileM = kPair ? 2 * kBM : kBM;
+  const int n_max = (kPair ? 2 : 1) * args.nbox_max * kBoxRows;   // rows per tile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -227,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
-      mbar_init(smem_u32(&tempty[a]), kEpiThreads);
+      mbar_init(smem_u32(&tempty[a]), (kPair ? 2 : 1) * kEpiWarps);   // one arrival per warp
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0u;
@@ -235,13 +299,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == kMmaWarp) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    if (kPair) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(kTmemCols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(kTmemCols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (kPair) cluster_sync();   // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // the prologue above overlaps the previous kernel; its outputs are read below
@@ -258,23 +330,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool issued[kMaxStages];
       for (int s = 0; s < kMaxStages; ++s) issued[s] = false, issued_parity[s] = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+      for (int t = unit; ok && t < n_tiles; t += n_units) {
         const Tile tl = tile_at(args, t);
         const int sd = (tl.g < args.E) ? 0 : 1;
         const Side& S = args.side[sd];
         const CUtensorMap* ma = sd ? &tmA1 : &tmA0;
         const CUtensorMap* mb = sd ? &tmB1 : &tmB0;
-        const int arow = (sd ? 0 : tl.g * S.m_rows) + tl.m0;
-        const int nmma = (tl.n + 15) & ~15;
-        int nbox = (nmma + kBoxRows - 1) / kBoxRows;
-        if (nbox > args.nbox_max) {   // never by construction; keeps the ring in bounds
+        const int arow = (sd ? 0 : tl.g * S.m_rows) + tl.m0 + (int)rank * kBM;
+        int nmma = (tl.n + 15) & ~15;
+        if (nmma > n_max) {   // never by construction; keeps the ring in bounds
           atomicOr(args.status, kStatusBadIndex);
-          nbox = args.nbox_max;
+          nmma = n_max;
         }
+        const int rows_here = kPair ? nmma / 2 : nmma;   // activation rows this CTA loads
+        const int brow = tl.r0 + (int)rank * rows_here;
+        const int nbox = (rows_here + kBoxRows - 1) / kBoxRows;
         // weight rows actually loaded: 128, or fewer for a gate matrix with
         // E < 128 rows (the other rows of the smem tile only feed outputs
         // that are never stored)
-        const uint32_t bytes = (uint32_t)S.a_rows * kBK * 2 + (uint32_t)nbox * kBoxBytes;
+        const uint32_t bytes_here = (uint32_t)S.a_rows * kBK * 2 + (uint32_t)nbox * kBoxBytes;
         const int kb0 = tl.ks * S.kb_per, kb1 = min(S.kb, kb0 + S.kb_per);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, args.status)) {
@@ -282,12 +356,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t fb = smem_u32(&full[stage]);
-          mbar_expect_tx(fb, bytes);
+          // the leader's barrier counts the bytes of both CTAs
+          if (leader) mbar_expect_tx(fb, (kPair ? 2u : 1u) * bytes_here);
           const uint32_t sa = smem_u32(ring + (size_t)stage * stage_bytes);
           const uint32_t sb = sa + kABytes;
-          tma_load_2d(sa, ma, kb * kBK, arow, fb);
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d(sb + i * kBoxBytes, mb, kb * kBK, tl.r0 + i * kBoxRows, fb);
+          if (kPair) {
+            const uint32_t fb0 = map_to_rank(fb, 0);
+            tma_load_2d_pair(sa, ma, kb * kBK, arow, fb0);
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d_pair(sb + i * kBoxBytes, mb, kb * kBK, brow + i * kBoxRows, fb0);
+          } else {
+            tma_load_2d(sa, ma, kb * kBK, arow, fb);
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d(sb + i * kBoxBytes, mb, kb * kBK, brow + i * kBoxRows, fb);
+          }
           issued[stage] = true;
           issued_parity[stage] = phase;
           if (++stage == n_stages) {
@@ -296,21 +378,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // every copy this thread started has landed before the CTA tears down
-      for (int s = 0; s < n_stages; ++s)
-        if (issued[s]) wait_bounded(smem_u32(&full[s]), issued_parity[s], nullptr, args.status);
+      // every copy started here has landed before the CTA pair tears down
+      // (the leader's barriers count the copies of both CTAs)
+      if (leader)
+        for (int s = 0; s < n_stages; ++s)
+          if (issued[s]) wait_bounded(smem_u32(&full[s]), issued_parity[s], nullptr, args.status);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+      for (int t = unit; ok && t < n_tiles; t += n_units) {
         const Tile tl = tile_at(args, t);
         const Side& S = args.side[(tl.g < args.E) ? 0 : 1];
-        const int nmma = min((tl.n + 15) & ~15, args.nbox_max * kBoxRows);
-        const uint32_t idesc = idesc_bf16(nmma);
+        const int nmma = min((tl.n + 15) & ~15, n_max);
+        const uint32_t idesc = idesc_bf16(nmma, kTileM);
         const int kb0 = tl.ks * S.kb_per, kb1 = min(S.kb, kb0 + S.kb_per);
         if (!wait_bounded(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
@@ -325,23 +409,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t adesc = sw128_desc(sa);
           const uint64_t bdesc = sw128_desc(sa + kABytes);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)   // 16 elements = 32 bytes per MMA
-            mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
-          mma_commit(smem_u32(&empty[stage]));
+          for (int k = 0; k < kBK / 16; ++k) {   // 16 elements = 32 bytes per MMA
+            const uint32_t accum = (kb != kb0 || k != 0) ? 1u : 0u;
+            if (kPair)
+              mma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+            else
+              mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+          }
+          if (kPair)
+            mma_commit_pair(smem_u32(&empty[stage]));
+          else
+            mma_commit(smem_u32(&empty[stage]));
           if (++stage == n_stages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(smem_u32(&tfull[acc]));
+        if (kPair)
+          mma_commit_pair(smem_u32(&tfull[acc]));
+        else
+          mma_commit(smem_u32(&tfull[acc]));
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
-      // retire every MMA this thread issued before TMEM is released
-      mma_commit(smem_u32(drain));
+      // retire every MMA issued before TMEM is released (in both CTAs)
+      if (kPair)
+        mma_commit_pair(smem_u32(drain));
+      else
+        mma_commit(smem_u32(drain));
+      wait_bounded(smem_u32(drain), 0, nullptr, args.status);
+    } else if (kPair && lane == 0) {
+      // the other CTA of the pair: its accumulators are written by the
+      // leader's MMAs; wait for the leader's final commit before release
       wait_bounded(smem_u32(drain), 0, nullptr, args.status);
     }
   } else {
@@ -352,8 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     const int quarter = warp & 3, half = warp >> 2;
-    const int row = quarter * 32 + lane;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int row = (int)rank * kBM + quarter * 32 + lane;
+    for (int t = unit; t < n_tiles; t += n_units) {
       const Tile tl = tile_at(args, t);
       const int sd = (tl.g < args.E) ? 0 : 1;
       const Side& S = args.side[sd];
@@ -368,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int col = tl.m0 + row;
       const bool store = col < S.m_valid;
       const size_t part = (size_t)tl.ks * (size_t)S.split_stride;
-      const int n = min(tl.n, args.nbox_max * kBoxRows);
+      const int n = min(tl.n, n_max);
       for (int c0 = half * 32; c0 < n; c0 += 64) {
         uint32_t r[32];
         __syncwarp();
@@ -390,7 +492,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&tempty[acc]));
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t te = smem_u32(&tempty[acc]);
+        if (kPair)
+          mbar_arrive_cluster(map_to_rank(te, 0));   // the leader reuses the accumulator
+        else
+          mbar_arrive(te);
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -400,10 +509,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (kPair) cluster_sync();   // no CTA of the pair leaves while the other may signal it
   if (warp == kMmaWarp) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(kTmemCols));
+    if (kPair)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(kTmemCols));
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(kTmemCols));
   }
 }
 
@@ -445,15 +559,19 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
 
 cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& shared, int E,
                                    bool gelu, const Tile* tiles, const int* n_tiles,
-                                   const DenseTiling* dense, uint32_t* status, int num_sms,
-                                   cudaStream_t st) {
+                                   const DenseTiling* dense, bool pair, uint32_t* status,
+                                   int num_sms, cudaStream_t st) {
   using namespace tc;
+  if (pair && dense) return cudaErrorInvalidValue;   // the gate GEMM runs single-CTA tiles
   static bool attr_set[64] = {false};   // per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(grouped_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(grouped_gemm_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(grouped_gemm_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
@@ -496,19 +614,24 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
   args.dense_splits = dense ? (routed.splits > 0 ? routed.splits : 1) : 1;
   // Ring shape: no tile has more rows than its activation matrix, so small
   // batches get small activation boxes per stage and a deeper ring (more
-  // weight bytes in flight per SM).
+  // weight bytes in flight per SM). A CTA of a pair loads half of the rows.
   uint64_t rows = routed.act_rows;
   if (shared.w) rows = std::max<uint64_t>(rows, shared.act_rows);
   const int max_n = (int)std::min<uint64_t>(kTcRows, (rows + 15) & ~15ull);
-  args.nbox_max = (max_n + kBoxRows - 1) / kBoxRows;
+  const int rows_per_cta = pair ? max_n / 2 : max_n;
+  args.nbox_max = std::max(1, (rows_per_cta + kBoxRows - 1) / kBoxRows);
   args.stage_bytes = kABytes + args.nbox_max * kBoxBytes;
   args.n_stages = std::min(kMaxStages, kStageArea / args.stage_bytes);
   args.status = status;
   args.E = E;
   args.gelu = gelu ? 1 : 0;
-  const int grid = dense ? std::min(num_sms, std::max(1, dense->tiles)) : num_sms;
-  return launch_pdl(grouped_gemm_tc, dim3(grid), dim3(kThreads), kSmemBytes, st, a0, b0, a1, b1,
-                    args);
+  if (!pair) {
+    const int grid = dense ? std::min(num_sms, std::max(1, dense->tiles)) : num_sms;
+    return launch_pdl(grouped_gemm_tc<false>, dim3(grid), dim3(kThreads), kSmemBytes, st, a0, b0,
+                      a1, b1, args);
+  }
+  return launch_pdl_cluster2(grouped_gemm_tc<true>, dim3(num_sms & ~1), dim3(kThreads),
+                             kSmemBytes, st, a0, b0, a1, b1, args);
 }
 
 }  // namespace moe

@@ -41,10 +41,12 @@ struct DenseTiling {
   int tiles, rows, m_tiles;
 };
 
+// pair: tiles of 256 weight rows on two-CTA clusters (tile list built with
+// 256-row weight blocks); otherwise 128 weight rows per CTA.
 cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& shared, int E,
                                    bool gelu, const Tile* tiles, const int* n_tiles,
-                                   const DenseTiling* dense, uint32_t* status, int num_sms,
-                                   cudaStream_t st);
+                                   const DenseTiling* dense, bool pair, uint32_t* status,
+                                   int num_sms, cudaStream_t st);
 
 cudaError_t launch_gate_logits(const moe_layer_desc& d, const void* x, const void* wr,
                                float* logits, cudaStream_t st);

@@ -226,7 +226,7 @@ cudaError_t launch_gate_logits_tc(const moe_layer_desc& d, const WsLayout& L, ch
   dense.m_tiles = (d.E + 127) / 128;
   dense.tiles = ((d.T + kTcRows - 1) / kTcRows) * dense.m_tiles * L.sp.router;
   return launch_grouped_gemm_tc(p, TcProblem{}, d.E, false, nullptr, nullptr, &dense,
-                                &hdr->status, num_sms, st);
+                                /*pair=*/false, &hdr->status, num_sms, st);
 }
 
 cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, int n_parts,
