@@ -347,3 +347,28 @@ def load_stats(counts: np.ndarray, T: int, K: int, cf_num: int = 5, cf_den: int 
         "num_stragglers": int(np.count_nonzero(c > cap)),
         "straggler_mask": (c > cap).astype(np.uint8),
     }
+
+
+# --------------------------------------------------------------------------
+# dynamic expert bias update (the other half of no-aux-loss routing)
+# --------------------------------------------------------------------------
+def bias_update(bias, counts, T: int, K: int, gamma: float, cf_num: int = 5, cf_den: int = 4):
+    """One low-frequency update of the expert bias B.
+
+    [K3-DIAG] 四: the bias B is updated rarely by a monitor; an expert that
+    stays overloaded has B_i lowered by a small step, one that stays idle has
+    it raised. Reading (the page gives neither step nor period): `counts` are
+    the expert loads accumulated over the caller's period and T the tokens of
+    that period; overloaded means count > capacity (capacity as in
+    load_stats), idle means count == 0; B_i -= gamma / += gamma, in fp32.
+    Returns the new bias as float32.
+    """
+    b = np.asarray(bias, dtype=np.float32).copy()
+    c = np.asarray(counts, dtype=np.int64)
+    cap = capacity(T, K, c.size, cf_num, cf_den)
+    g = np.float32(gamma)
+    over = c > cap
+    idle = c == 0
+    b[over] = (b[over] - g).astype(np.float32)
+    b[idle] = (b[idle] + g).astype(np.float32)
+    return b

@@ -377,3 +377,34 @@ def test_combine_K1_unit_weight_is_inverse_permutation():
     inv[perm] = np.arange(TK)
     y = oracle.combine(rows, np.ones((TK, 1)), inv)
     np.testing.assert_array_equal(y, rows[inv])
+
+
+# ------------------------------------------------------------ bias update ---
+def test_bias_update_moves_only_overloaded_and_idle_experts():
+    counts = np.array([30, 0, 5, 10, 0, 11])           # T=16, K=3, E=6: capacity = 48*5//24 = 10
+    b = np.array([0.0, 0.5, -0.25, 1.0, 0.0, -1.0], np.float32)
+    nb = oracle.bias_update(b, counts, 16, 3, 0.125)
+    assert oracle.capacity(16, 3, 6) == 10
+    assert nb.tolist() == [-0.125, 0.625, -0.25, 1.0, 0.125, -1.125]
+    assert nb.dtype == np.float32
+
+
+def test_bias_update_is_a_fixed_point_for_an_even_load():
+    counts = np.full(16, 8)
+    b = np.linspace(-1, 1, 16).astype(np.float32)
+    assert (oracle.bias_update(b, counts, 64, 2, 0.01) == b).all()
+
+
+def test_repeated_bias_updates_even_out_a_skewed_router():
+    """The page's stated purpose: routing with the updated bias spreads the
+    load (Gini falls) without retraining the gate."""
+    rng = _rng(51)
+    T, E, K = 512, 32, 4
+    logits = rng.normal(size=(T, E)) - 0.6 * np.log(np.arange(E) + 1.0)
+    b = np.zeros(E, np.float32)
+    g0 = oracle.gini_exact(oracle.expert_counts(oracle.select_topk(logits, b, K)[0], E))
+    for _ in range(60):
+        counts = oracle.expert_counts(oracle.select_topk(logits, b, K)[0], E)
+        b = oracle.bias_update(b, counts, T, K, 0.02)
+    g1 = oracle.gini_exact(oracle.expert_counts(oracle.select_topk(logits, b, K)[0], E))
+    assert g1 < 0.6 * g0
