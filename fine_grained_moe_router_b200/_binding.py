@@ -23,7 +23,7 @@ MOE_F32, MOE_BF16 = 0, 1
 EXPORTED = (
     "moe_workspace_size", "moe_router_topk", "moe_topk_from_logits", "moe_dispatch",
     "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
-    "moe_expert_stats",
+    "moe_expert_stats", "moe_bias_update",
     "moe_check_status", "moe_status_string", "moe_kernel_launch_count", "moe_dispatch_noalloc",
 )
 
@@ -77,6 +77,7 @@ def _load() -> ctypes.CDLL:
                                                       ctypes.POINTER(MoERouting), P, S, P,
                                                       ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
         "moe_expert_stats": (ctypes.c_int, [D, P, P, ctypes.POINTER(MoEStats), P, S, P]),
+        "moe_bias_update": (ctypes.c_int, [D, P, P, ctypes.c_float, P]),
         "moe_check_status": (ctypes.c_int, [P, S, P]),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_kernel_launch_count": (ctypes.c_uint64, []),
@@ -216,6 +217,12 @@ def moe_expert_stats(desc, counts, straggler_mask, ws, stream=None) -> dict:
                                 ctypes.byref(out), _p(ws), ws.numel() if ws is not None else 0,
                                 _stream(stream)), "moe_expert_stats")
     return out.as_dict()
+
+
+def moe_bias_update(desc, counts, bias, gamma: float, stream=None) -> None:
+    """Updates `bias` [E] fp32 in place from the accumulated `counts` [E] int32."""
+    _check(lib.moe_bias_update(ctypes.byref(desc), _p(counts), _p(bias), ctypes.c_float(gamma),
+                               _stream(stream)), "moe_bias_update")
 
 
 def moe_kernel_launch_count() -> int:

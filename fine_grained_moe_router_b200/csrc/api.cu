@@ -2,6 +2,7 @@
 // Every compute step runs in this library's kernels; nothing here computes
 // on the host except sizes.
 #include <atomic>
+#include <cmath>
 #include <cstring>
 
 #include "common.cuh"
@@ -409,6 +410,15 @@ moe_status moe_expert_stats(const moe_layer_desc* desc, const int32_t* counts,
   MOE_CUDA_TRY(launch_expert_stats(d, counts, straggler_mask_or_null, dev, st));
   MOE_CUDA_TRY(cudaMemcpyAsync(out_host, dev, sizeof(moe_stats), cudaMemcpyDeviceToHost, st));
   MOE_CUDA_TRY(cudaStreamSynchronize(st));
+  return MOE_OK;
+}
+
+moe_status moe_bias_update(const moe_layer_desc* desc, const int32_t* counts, float* bias,
+                           float gamma, moe_stream stream) {
+  MOE_TRY(check_desc(desc));
+  if (!counts || !bias) return MOE_ERR_INVALID_ARG;
+  if (!(gamma >= 0.f) || !std::isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(launch_bias_update(*desc, counts, bias, gamma, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 

@@ -208,4 +208,32 @@ cudaError_t launch_expert_stats(const moe_layer_desc& d, const int32_t* counts, 
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Dynamic expert bias update ("Kimi K3 专家路由不均衡诊断" §四): an expert that
+// stayed overloaded over the caller's period (accumulated count > capacity)
+// has its bias lowered by gamma, an idle one (count == 0) raised by gamma,
+// in fp32; the others keep theirs.
+__global__ void __launch_bounds__(512) bias_update_kernel(const int32_t* __restrict__ counts,
+                                                          float* __restrict__ bias, int E,
+                                                          long long capacity, float gamma) {
+  pdl_wait();
+  pdl_trigger();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const long long c = counts[e];
+    float b = bias[e];
+    if (c > capacity)
+      b = __fsub_rn(b, gamma);
+    else if (c == 0)
+      b = __fadd_rn(b, gamma);
+    bias[e] = b;
+  }
+}
+
+cudaError_t launch_bias_update(const moe_layer_desc& d, const int32_t* counts, float* bias,
+                               float gamma, cudaStream_t st) {
+  const long long TK = (long long)d.T * d.K;
+  const long long cap = TK * d.cf_num / ((long long)d.E * d.cf_den);
+  return launch_pdl(bias_update_kernel, dim3(1), dim3(512), 0, st, counts, bias, d.E, cap, gamma);
+}
+
 }  // namespace moe

@@ -78,6 +78,8 @@ cudaError_t launch_grouped_gemm_simt(int dtype, bool gelu, const SimtProblem& ro
 cudaError_t launch_combine(const moe_layer_desc& d, const void* y_rows, const float* w,
                            const int32_t* inv, const void* y_shared, void* y, cudaStream_t st,
                            int rows_parts = 1, int shared_parts = 1);
+cudaError_t launch_bias_update(const moe_layer_desc& d, const int32_t* counts, float* bias,
+                               float gamma, cudaStream_t st);
 cudaError_t launch_expert_stats(const moe_layer_desc& d, const int32_t* counts, uint8_t* mask,
                                 moe_stats* out_dev, cudaStream_t st);
 

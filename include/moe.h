@@ -199,7 +199,11 @@ moe_status moe_combine(const moe_layer_desc* desc, const void* y_rows, const flo
                        moe_stream stream);
 
 /* The whole layer: router, dispatch, grouped FFN (+ shared), combine.
- * y [T, H]. routing_or_null: optional copies of the routing tensors. */
+ * y [T, H]. routing_or_null: optional copies of the routing tensors.
+ * Every launch goes to `stream`, and no host decision depends on device
+ * data, so the call can be captured into a CUDA graph and replayed (the
+ * graph keeps the pointers and the shape of the captured call). The first
+ * call for a device must run outside capture: it sets kernel attributes. */
 moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* weights,
                              const void* x, void* y, const moe_routing* routing_or_null,
                              void* ws, size_t ws_bytes, moe_stream stream);
@@ -224,6 +228,19 @@ moe_status moe_layer_forward_profiled(const moe_layer_desc* desc,
 moe_status moe_expert_stats(const moe_layer_desc* desc, const int32_t* counts,
                             uint8_t* straggler_mask_or_null, moe_stats* out_host, void* ws,
                             size_t ws_bytes, moe_stream stream);
+
+/* Dynamic expert bias update, the monitor side of no-aux-loss routing:
+ * "Kimi K3 专家路由不均衡诊断" §四 (an expert that stays overloaded has its
+ * bias B_i lowered by a small step, one that stays idle has it raised).
+ *   counts [E] int32 (device): expert loads accumulated over the caller's
+ *   update period; desc->T: the tokens of that period (with K, E and the
+ *   capacity factor it sets capacity = floor(T*K*cf_num / (E*cf_den)));
+ *   bias [E] fp32 (device, updated in place): B_e -= gamma where
+ *   counts[e] > capacity, B_e += gamma where counts[e] == 0, in fp32.
+ * Asynchronous on `stream`; the next moe_layer_forward on the stream sees
+ * the new bias. */
+moe_status moe_bias_update(const moe_layer_desc* desc, const int32_t* counts, float* bias,
+                           float gamma, moe_stream stream);
 
 /* Reads and clears the workspace status word (synchronises `stream`):
  * MOE_OK, or MOE_ERR_TIMEOUT if a bounded device wait ran out. */
