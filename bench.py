@@ -307,6 +307,25 @@ class Runner:
         ms = max_over_ranks(start.elapsed_time(end), world, device)
         return ms, launches
 
+    def timed_graph(self, steps, warmup):
+        """The same forward captured once in a CUDA graph and replayed."""
+        self.step()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step()
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(steps):
+            g.replay()
+        end.record()
+        torch.cuda.synchronize()
+        del g
+        return start.elapsed_time(end)
+
     def stages(self, steps):
         """Per-stage device times (ms, mean over steps) from events recorded
         between the kernels of moe_layer_forward_profiled."""
@@ -430,7 +449,9 @@ def measure_point(M, wl, dev, T, peaks, steps=20, warmup=5):
     alg = algorithmic(wl, T, R.touched())
     bound, t_roof = roofline_bound(alg["flops"], alg["bytes"], peaks)
     ms_step = ms / steps
+    graph_ms = R.timed_graph(steps, warmup) / steps
     return {"workload": wl.key, "T": T, "tokens_per_s": T / (ms_step / 1e3), "us_per_step": 1e3 * ms_step,
+            "graph_us_per_step": 1e3 * graph_ms, "graph_frac": 1e3 * t_roof / graph_ms,
             "bound": bound, "roofline_us": 1e6 * t_roof, "frac": 1e3 * t_roof / ms_step,
             "experts_touched": R.touched(), "stages_us": {k: 1e3 * v for k, v in st.items()}}
 
