@@ -211,6 +211,30 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 32 lanes x 64 consecutive fp32 columns of the accumulator (one register
+// per column), waited for before returning.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+        "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 struct Side {          // routed experts (0) or the shared expert (1)
   void* out;           // output rows, row stride `ld` elements
   long long split_stride;   // elements between the partial outputs of two splits
@@ -249,6 +273,50 @@ __device__ __forceinline__ Tile tile_at(const Args& a, int t) {
   tl.n = min(kTcRows, a.dense_rows - tl.r0);
   tl.g = 0;
   return tl;
+}
+
+// Epilogue of one accumulator for the warp's TMEM lane quarter. Thread = one
+// output column (o0 = its offset in output row tl.r0); accumulator column j
+// goes to output row tl.r0 + j. The two warps of a quarter take alternate
+// chunks of kW columns (kW = 64 for plain stores, 32 with the GeLU, whose
+// temporaries need the registers). The output mode is a template
+// parameter, so the per-element loop carries no branches.
+enum EpiMode { kEpiF32 = 0, kEpiBf16 = 1, kEpiGeluBf16 = 2 };
+
+template <int kW>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[kW]) {
+  if constexpr (kW == 64)
+    tmem_ld64(taddr, r);
+  else
+    tmem_ld32(taddr, r);
+}
+
+template <int kMode, int kW>
+__device__ __forceinline__ void epilogue_columns(uint32_t taddr, int half, int n, bool store,
+                                                 void* out, size_t o0, int ld) {
+  for (int c0 = half * kW; c0 < n; c0 += 2 * kW) {
+    uint32_t r[kW];
+    __syncwarp();
+    tmem_ld_cols<kW>(taddr + (uint32_t)c0, r);
+    if (!store) continue;
+    const int cnt = min(kW, n - c0);
+    const size_t o = o0 + (size_t)c0 * (size_t)ld;
+    if (kMode == kEpiF32) {
+      float* p = static_cast<float*>(out) + o;
+#pragma unroll
+      for (int q = 0; q < kW; ++q)
+        if (q < cnt) p[(size_t)q * ld] = __uint_as_float(r[q]);
+    } else {
+      __nv_bfloat16* p = static_cast<__nv_bfloat16*>(out) + o;
+#pragma unroll
+      for (int q = 0; q < kW; ++q)
+        if (q < cnt) {
+          float v = __uint_as_float(r[q]);
+          if (kMode == kEpiGeluBf16) v = gelu_erf(v);
+          p[(size_t)q * ld] = __float2bfloat16_rn(v);
+        }
+    }
+  }
 }
 
 // kPair = false: one CTA per tile of 128 weight rows (MMA M = 128).
@@ -449,8 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // --------------------------------------------------------- epilogue
     // warp w reads TMEM lanes 32*(w%4) .. +31 (thread = weight row of the
-    // tile) and the 32-column chunks (w/4), (w/4)+2, ... of the accumulator
-    // (column = activation row of the tile).
+    // tile) and every other column chunk of the accumulator, starting at
+    // chunk w/4 (column = activation row of the tile).
     int acc = 0;
     uint32_t acc_phase = 0;
     const int quarter = warp & 3, half = warp >> 2;
@@ -471,26 +539,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool store = col < S.m_valid;
       const size_t part = (size_t)tl.ks * (size_t)S.split_stride;
       const int n = min(tl.n, n_max);
-      for (int c0 = half * 32; c0 < n; c0 += 64) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld32(taddr + (uint32_t)c0, r);
-        if (store) {
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int j = c0 + q;
-            if (j < n) {
-              float v = __uint_as_float(r[q]);
-              if (args.gelu) v = gelu_erf(v);
-              const size_t o = part + (size_t)(tl.r0 + j) * S.ld + col;
-              if (S.out_f32)
-                static_cast<float*>(S.out)[o] = v;
-              else
-                static_cast<__nv_bfloat16*>(S.out)[o] = __float2bfloat16_rn(v);
-            }
-          }
-        }
-      }
+      const size_t o0 = part + (size_t)tl.r0 * (size_t)S.ld + (size_t)col;
+      if (args.gelu)
+        epilogue_columns<kEpiGeluBf16, 32>(taddr, half, n, store, S.out, o0, S.ld);
+      else if (S.out_f32)
+        epilogue_columns<kEpiF32, 64>(taddr, half, n, store, S.out, o0, S.ld);
+      else
+        epilogue_columns<kEpiBf16, 64>(taddr, half, n, store, S.out, o0, S.ld);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

@@ -107,23 +107,39 @@ __device__ __forceinline__ void select_row(const float* __restrict__ lrow, int n
                                            float* __restrict__ w_out,
                                            float* __restrict__ logits_out) {
   const int lane = threadIdx.x & 31;
+  // Sum of the n_parts partial logits (reduction splits of the gate GEMM)
+  // in split order. The loads of kPB parts for all NJ slots are issued
+  // before any add, so the partial sums cost one round trip per kPB parts.
+  constexpr int kPB = (NJ >= 8) ? 4 : (NJ >= 4 ? 8 : 16);
+  float l[NJ];
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int e = lane + 32 * j;
+    l[j] = (e < E) ? lrow[e] : 0.f;
+  }
+  for (int p0 = 1; p0 < n_parts; p0 += kPB) {
+    float v[kPB][NJ];
+#pragma unroll
+    for (int q = 0; q < kPB; ++q)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int e = lane + 32 * j;
+        v[q][j] = (p0 + q < n_parts && e < E) ? lrow[(p0 + q) * part_stride + e] : 0.f;
+      }
+#pragma unroll
+    for (int q = 0; q < kPB; ++q)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j)
+        if (p0 + q < n_parts) l[j] = __fadd_rn(l[j], v[q][j]);
+  }
   float s[NJ];
 #pragma unroll
   for (int j = 0; j < NJ; ++j) {
     const int e = lane + 32 * j;
     if (e < E) {
-      float l = lrow[e];
-      for (int p0 = 1; p0 < n_parts; p0 += 8) {   // 8 independent loads, then in-order adds
-        float v[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = (p0 + q < n_parts) ? lrow[(p0 + q) * part_stride + e] : 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (p0 + q < n_parts) l = __fadd_rn(l, v[q]);
-      }
-      if (logits_out) logits_out[e] = l;
+      if (logits_out) logits_out[e] = l[j];
       const float b = bias ? bias[e] : 0.f;
-      s[j] = __fadd_rn(l, b);
+      s[j] = __fadd_rn(l[j], b);
     } else {
       s[j] = -INFINITY;
     }
