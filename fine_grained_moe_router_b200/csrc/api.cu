@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -18,11 +19,9 @@ size_t dtype_size(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
 static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Reduction splits for the tensor-core GEMMs. A decode-sized step has too
-// few (128-row x all-K) tiles to give every one of the 148 SMs a share of
-// the weight stream; splitting the reduction multiplies the tiles. The
-// choice depends on the shape only (so the workspace size does too):
-// about kTargetTiles tiles, at least 2 (router) or 4 (expert GEMM) reduction
-// blocks per split, and no empty split.
+// few (128-row x all-K) tiles to give every one of the 148 SMs an equal share
+// of the weight stream; splitting the reduction multiplies the tiles. The
+// choice depends on the shape only (so the workspace size does too).
 static int split_count(long long tiles, int kb, int want_tiles, int min_kb) {
   if (tiles <= 0 || tiles >= want_tiles) return 1;
   int sp = (int)((want_tiles + tiles - 1) / tiles);
@@ -32,8 +31,72 @@ static int split_count(long long tiles, int kb, int want_tiles, int min_kb) {
   return (kb + per - 1) / per;
 }
 
-Splits choose_splits(const moe_layer_desc& d) {
-  Splits s{1, 1, 1, 0};
+// Splits that leave no empty split: kb blocks in ceil(kb / ceil(kb / sp)).
+static int normalise_splits(int kb, int sp) {
+  const int per = (kb + sp - 1) / sp;
+  return (kb + per - 1) / per;
+}
+
+// Largest share of one persistent unit, in reduction blocks, when ns tiles
+// of cost cs and then nr tiles of cost cr are dealt round-robin to `units`
+// units: the order of the device tile list when every touched expert has one
+// row tile (the shared expert's tiles come first).
+static double deal_makespan(long long ns, double cs, long long nr, double cr, int units) {
+  double worst = 0.0;
+  const long long n = ns + nr;
+  for (int u = 0; u < units && u < n; ++u) {
+    const long long k_all = (n - u + units - 1) / units;
+    const long long k_sh = ns > u ? (ns - u + units - 1) / units : 0;
+    worst = std::max(worst, (double)k_sh * cs + (double)(k_all - k_sh) * cr);
+  }
+  return worst;
+}
+
+// Splits (routed, shared) of one weight-streaming GEMM launch with ns shared
+// tiles of kbs reduction blocks and nr_lo .. nr_hi routed tiles of kbr blocks
+// (the routed count depends on how many experts the batch touches, which
+// the shape alone does not fix). Each candidate is scored by its per-unit
+// share relative to a perfect spread, averaged over the low, middle and high
+// routed counts; each tile also costs tile_cost blocks of fixed work, and
+// near-ties go to fewer splits. At most max_r / max_s splits and at least
+// kMinKb blocks per split.
+static void pick_splits(long long nr_lo, long long nr_hi, int kbr, long long ns, int kbs,
+                        int units, int max_r, int max_s, double tile_cost, int* sr_out,
+                        int* ss_out) {
+  constexpr int kMinKb = 4;
+  static const int kCand[] = {1, 2, 3, 4, 5, 6, 8, 10, 12, 16};
+  const long long nr_at[3] = {nr_lo, (nr_lo + nr_hi) / 2, nr_hi};
+  double best = 1e300;
+  int br = 1, bs = 1;
+  for (int cr : kCand) {
+    if (cr > 1 && (cr > max_r || kbr / cr < kMinKb)) break;
+    const int sr = normalise_splits(kbr, cr);
+    for (int cs : kCand) {
+      if (cs > 1 && (ns == 0 || cs > max_s || kbs / cs < kMinKb)) break;
+      const int ss = normalise_splits(kbs > 0 ? kbs : 1, cs);
+      const double per_r = (double)((kbr + sr - 1) / sr);
+      const double per_s = kbs ? (double)((kbs + ss - 1) / ss) : 0.0;
+      double score = 0.0;
+      for (long long nr : nr_at) {
+        const double ideal =
+            std::max(1.0, ((double)ns * kbs + (double)nr * kbr) / (double)units);
+        score += deal_makespan(ns * ss, per_s + tile_cost, nr * sr, per_r + tile_cost, units) /
+                 ideal;
+      }
+      score *= 1.0 + 0.01 * (sr + ss - 2);
+      if (score < best * 0.999) {
+        best = score;
+        br = sr;
+        bs = ss;
+      }
+    }
+  }
+  *sr_out = br;
+  *ss_out = bs;
+}
+
+static Splits compute_splits(const moe_layer_desc& d) {
+  Splits s{1, 1, 1, 1, 1, 0};
   if (d.dtype != MOE_BF16 || d.T == 0) return s;
   const long long T = d.T, TK = (long long)d.T * d.K;
   // CTA pairs (256 weight rows per tile) when the touched experts average
@@ -41,17 +104,36 @@ Splits choose_splits(const moe_layer_desc& d) {
   // halved per-SM operand traffic to matter.
   const long long touched = std::min<long long>(d.E, TK);
   s.pair = (d.D % 256 == 0 && d.H % 256 == 0 && d.Ds % 256 == 0 && TK >= 64 * touched) ? 1 : 0;
-  const int kTargetTiles = s.pair ? 148 : 296;   // two per SM or per pair
   const long long row_tiles = (T + kTcRows - 1) / kTcRows;
   s.router = std::min(16, split_count(row_tiles * ((d.E + 127) / 128), d.H / 64, 148, 2));
-  {  // no empty split after the cap
-    const int kb = d.H / 64, per = (kb + s.router - 1) / s.router;
-    s.router = (kb + per - 1) / per;
+  s.router = normalise_splits(d.H / 64, s.router);   // no empty split after the cap
+  // Each touched expert has at least one row tile; a decode step touches
+  // min(E, T*K) experts.
+  const long long r_rows = std::max(touched, (TK + kTcRows - 1) / kTcRows);
+  if (!s.pair) {
+    // Weight-streaming regime: balance both expert GEMMs over the SMs. The
+    // first GEMM's splits are added up by the last split of each tile, one
+    // round of loads per few rows, so they are used for short tiles only:
+    // at most kFixupRows rows per routed expert on average, or per shared tile.
+    constexpr int kFixupRows = 16;
+    const int max_r1 = (TK <= kFixupRows * touched) ? 16 : 1;
+    const int max_s1 = (T <= kFixupRows) ? 16 : 1;
+    // Fixed cost per tile, in reduction blocks: the first layer's splits
+    // also pay the partial round trip and the fixup.
+    // a batch touches between K and min(E, T*K) experts
+    const long long r_lo = std::max<long long>(d.K + (touched - d.K) / 2, (TK + kTcRows - 1) / kTcRows);
+    pick_splits(r_lo * (d.D / 128), r_rows * (d.D / 128), d.H / 64,
+                d.Ds ? row_tiles * (d.Ds / 128) : 0, d.H / 64, 148, max_r1, max_s1, 6.0,
+                &s.gemm1_routed, &s.gemm1_shared);
+    pick_splits(r_lo * (d.H / 128), r_rows * (d.H / 128), d.D / 64,
+                d.Ds ? row_tiles * (d.H / 128) : 0, d.Ds ? d.Ds / 64 : 0, 148, 16, 16, 2.0,
+                &s.gemm2_routed, &s.gemm2_shared);
+    return s;
   }
-  // GEMM2: each touched expert has at least one row tile; a decode step
-  // touches min(E, T*K) experts.
-  const int mt2 = d.H / (s.pair ? 256 : 128);
-  const long long r_tiles = std::max(std::min<long long>(d.E, TK), (TK + kTcRows - 1) / kTcRows) * mt2;
+  // CTA pairs: split the second GEMM only when it has fewer tiles than pairs
+  constexpr int kTargetTiles = 148;
+  const int mt2 = d.H / 256;
+  const long long r_tiles = r_rows * mt2;
   const long long s_tiles = d.Ds ? row_tiles * mt2 : 0;
   if (r_tiles + s_tiles < kTargetTiles) {
     const int kbr = d.D / 64, kbs = d.Ds / 64;
@@ -60,6 +142,29 @@ Splits choose_splits(const moe_layer_desc& d) {
     s.gemm2_routed = split_count(1, kbr, (kbr + per - 1) / per, 4);
     if (d.Ds) s.gemm2_shared = split_count(1, kbs, (kbs + per - 1) / per, 4);
   }
+  return s;
+}
+
+// The choice is a pure function of the descriptor; a small cache keeps its
+// search off the per-call host path.
+Splits choose_splits(const moe_layer_desc& d) {
+  struct Entry {
+    moe_layer_desc d;
+    Splits s;
+    bool used;
+  };
+  static std::mutex mu;
+  static Entry cache[16] = {};
+  static int next = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : cache)
+      if (e.used && std::memcmp(&e.d, &d, sizeof(d)) == 0) return e.s;
+  }
+  const Splits s = compute_splits(d);
+  std::lock_guard<std::mutex> lock(mu);
+  cache[next] = Entry{d, s, true};
+  next = (next + 1) % 16;
   return s;
 }
 
@@ -75,7 +180,8 @@ WsLayout workspace_layout(const moe_layer_desc& d) {
   const size_t rt_routed = (TK + kTcRows - 1) / kTcRows + rows_bound;
   const size_t rt_shared = Ds ? (T + kTcRows - 1) / kTcRows : 0;
   L.sp = choose_splits(d);
-  L.max_tiles_tc1 = (int)(rt_routed * (D / 128) + rt_shared * (Ds / 128));
+  L.max_tiles_tc1 =
+      (int)((rt_routed * L.sp.gemm1_routed * (D / 128) + rt_shared * L.sp.gemm1_shared * (Ds / 128)));
   L.max_tiles_tc2 =
       (int)((rt_routed * L.sp.gemm2_routed + rt_shared * L.sp.gemm2_shared) * (H / 128));
   size_t o = 0;
@@ -101,6 +207,9 @@ WsLayout workspace_layout(const moe_layer_desc& d) {
   L.xp = take(d.dtype == MOE_BF16 ? es * TK * H : 0);
   L.hm = take(es * TK * D);
   L.hs = take(es * T * Ds);
+  // fp32 partial outputs of the first GEMM when its reduction is split
+  L.p1r = take(L.sp.gemm1_routed > 1 ? sizeof(float) * TK * D * L.sp.gemm1_routed : 0);
+  L.p1s = take(Ds && L.sp.gemm1_shared > 1 ? sizeof(float) * T * Ds * L.sp.gemm1_shared : 0);
   // expert outputs are fp32, one copy per reduction split of the second GEMM
   L.yr = take(sizeof(float) * TK * H * L.sp.gemm2_routed);
   L.ys = take(sizeof(float) * T * H * (Ds ? L.sp.gemm2_shared : 0));
@@ -190,12 +299,25 @@ static moe_status run_grouped_ffn(const moe_layer_desc& d, const WsLayout& L, ch
       return p;
     };
     const int sp_r = split ? L.sp.gemm2_routed : 1, sp_s = split ? L.sp.gemm2_shared : 1;
+    const int sp1_r = split ? L.sp.gemm1_routed : 1, sp1_s = split ? L.sp.gemm1_shared : 1;
+    // A split first layer writes fp32 partials; the last split of each tile
+    // to finish adds them and writes the GeLU output.
+    auto split_first_layer = [](TcProblem& p, void* partials, int splits, long long rows) {
+      p.fix_out = p.out;
+      p.fix_ld = p.ld;
+      p.out = partials;
+      p.out_f32 = true;
+      p.splits = splits;
+      p.split_stride = rows * p.ld;
+    };
     TcProblem r1 = problem(ws + L.xp, TK, w1, (uint64_t)d.E * d.D, d.D, d.H, hm, d.D, false, 1, 0);
+    if (sp1_r > 1) split_first_layer(r1, ws + L.p1r, sp1_r, (long long)TK);
     TcProblem r2 = problem(hm, TK, w2, (uint64_t)d.E * d.H, d.H, d.D, y_rows, d.H, true, sp_r,
                            (long long)TK * d.H);
     TcProblem s1{}, s2{};
     if (shared) {
       s1 = problem(x, (uint64_t)d.T, ws1, (uint64_t)d.Ds, d.Ds, d.H, hs, d.Ds, false, 1, 0);
+      if (sp1_s > 1) split_first_layer(s1, ws + L.p1s, sp1_s, (long long)d.T);
       s2 = problem(hs, (uint64_t)d.T, ws2, (uint64_t)d.H, d.H, d.Ds, y_shared, d.H, true, sp_s,
                    (long long)d.T * d.H);
     }

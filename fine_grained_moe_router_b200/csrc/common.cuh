@@ -51,15 +51,24 @@ struct Tile {
   int32_t n;
   int32_t m0;   // first output column (weight row) of the tile; used by the tensor-core path
   int32_t ks;   // reduction split of the tile (tensor-core path), 0 when unsplit
-  int32_t pad[3];
+  // First-layer tiles with reduction splits: in the split-0 tile, arrival
+  // counters of the tile's splits for the CTA (or each CTA of a pair);
+  // in every split, the list index of its split-0 tile. Written as 0 / the
+  // index by the dispatch step each forward.
+  int32_t arrivals[2];
+  int32_t first_split;
 };
 
 // Reduction splits of the tensor-core GEMMs of one layer forward (chosen on
 // the host from the shape alone). A split s of a tile covers reduction blocks
-// [s * kb_per, (s + 1) * kb_per) and writes its own fp32 partial output; the
-// consumer kernel adds the partials in split order.
+// [s * kb_per, (s + 1) * kb_per) and writes its own fp32 partial output. The
+// partials are added in split order: by the selection kernel (gate GEMM), by
+// the last split of a tile to finish (first expert layer, before its GeLU),
+// or by the combine kernel (second expert layer).
 struct Splits {
   int router;        // gate GEMM
+  int gemm1_routed;  // first expert layer, routed experts
+  int gemm1_shared;  // first expert layer, shared expert
   int gemm2_routed;  // second expert layer, routed experts
   int gemm2_shared;  // second expert layer, shared expert
   int pair;          // 1: expert GEMMs on CTA pairs (256 weight rows per tile)
@@ -68,7 +77,7 @@ struct Splits {
 // Offsets of each workspace region (bytes), 256-byte aligned.
 struct WsLayout {
   size_t hdr, hist, base, tiles_simt, tiles_tc1, tiles_tc2, idx, w, counts, offsets, perm, inv,
-      logits, logits_part, xp, hm, hs, yr, ys, stats, total;
+      logits, logits_part, xp, hm, hs, p1r, p1s, yr, ys, stats, total;
   int n_chunks;
   int max_tiles_simt, max_tiles_tc1, max_tiles_tc2;
   Splits sp;

@@ -78,6 +78,7 @@ struct TileSpec {
   Tile* tc2;           // tensor-core tiles of GEMM2
   int m_tiles1_routed, m_tiles1_shared;   // output-column tiles (128 wide) of GEMM1
   int m_tiles2;                           // output-column tiles of GEMM2 (H / 128)
+  int splits1_routed, splits1_shared;     // reduction splits of GEMM1 tiles
   int splits2_routed, splits2_shared;     // reduction splits of GEMM2 tiles
   int mtile;                              // weight rows per tile: 128, or 256 on CTA pairs
 };
@@ -120,12 +121,10 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
     }
   }
   // Tensor-core tiles: balanced row blocks (<= kTcRows rows, multiple of 16)
-  // times 128-wide weight-row blocks. Order: the shared expert first, then
-  // the routed experts by descending row count (ties by index), so the
-  // longest work starts first; inside a group the weight-row blocks are
-  // outermost and the row blocks innermost, so the row blocks that share a
-  // 128-row weight slab run at the same time on neighbouring CTAs and read
-  // the slab from L2 instead of DRAM.
+  // times weight-row blocks (128, or 256 on CTA pairs) times reduction
+  // splits. Order: the shared expert first, then the routed experts by
+  // descending row count (ties by index), so the longest work starts first;
+  // the order inside a group is given where the tiles are written.
   __shared__ int s_cnt[kMaxE];
   __shared__ int s_pos1[kMaxE], s_pos2[kMaxE];
   __shared__ int s_first1[kMaxE + 1], s_first2[kMaxE + 1], s_nt[kMaxE + 1], s_rper[kMaxE + 1],
@@ -135,7 +134,8 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
   const int mt1 = (e < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared;
   int sh_nt, sh_rper;
   tc_row_split(has_shared ? T : 0, &sh_nt, &sh_rper);
-  const int sh1 = sh_nt * ts.m_tiles1_shared, sh2 = sh_nt * ts.m_tiles2 * ts.splits2_shared;
+  const int sh1 = sh_nt * ts.m_tiles1_shared * ts.splits1_shared;
+  const int sh2 = sh_nt * ts.m_tiles2 * ts.splits2_shared;
   if (e < E) s_cnt[e] = c;
   __syncthreads();
   int rank = 0;
@@ -144,7 +144,7 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
       const int cq = s_cnt[q];
       rank += (cq > c) || (cq == c && q < e);
     }
-    s_pos1[rank] = nt_rows * mt1;                  // tile counts in rank order
+    s_pos1[rank] = nt_rows * mt1 * ts.splits1_routed;   // tile counts in rank order
     s_pos2[rank] = nt_rows * ts.m_tiles2 * ts.splits2_routed;
   }
   __syncthreads();
@@ -171,20 +171,22 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
       const int nt = s_nt[g];
       if (nt == 0) continue;
       const int m1 = (g < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared;
+      const int sp1 = (g < E) ? ts.splits1_routed : ts.splits1_shared;
       const int sp2 = (g < E) ? ts.splits2_routed : ts.splits2_shared;
-      const int n1 = nt * m1, n2 = nt * ts.m_tiles2 * sp2;
+      const int n1 = nt * m1 * sp1, n2 = nt * ts.m_tiles2 * sp2;
       for (int i = lane; i < n1 + n2; i += 32) {
         const bool first = i < n1;
         const int j = first ? i : i - n1;
-        const int sp = first ? 1 : sp2;
+        const int sp = first ? sp1 : sp2;
         const int mt = first ? m1 : ts.m_tiles2;
         // Order inside the group: when the group has more activation rows than
         // weight rows the row blocks are outermost (the weight matrix stays in
         // L2 while the rows stream once); otherwise the weight blocks are
         // outermost (each weight slab streams once while its row blocks, on
         // neighbouring CTAs, reuse it from L2). Splits vary fastest after that.
-        int r, q;
-        if (s_rows[g] > mt * ts.mtile) {
+        int r, q, j0;   // j0: the list position of the split-0 tile of j
+        const bool row_outer = s_rows[g] > mt * ts.mtile;
+        if (row_outer) {
           r = j / (mt * sp);
           q = j - r * (mt * sp);
         } else {
@@ -197,10 +199,16 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
         t.n = min(s_rper[g], s_rows[g] - r * s_rper[g]);
         t.m0 = (q / sp) * ts.mtile;
         t.ks = q % sp;
-        if (first)
+        j0 = row_outer ? j - t.ks : j - t.ks * nt;
+        t.arrivals[0] = 0;
+        t.arrivals[1] = 0;
+        if (first) {
+          t.first_split = s_first1[g] + j0;
           ts.tc1[s_first1[g] + j] = t;
-        else
+        } else {
+          t.first_split = s_first2[g] + j0;
           ts.tc2[s_first2[g] + j] = t;
+        }
       }
     }
   }
@@ -325,16 +333,13 @@ __global__ void __launch_bounds__(256) chunk_scatter(const int32_t* __restrict__
 // (warp, expert) live in dynamic shared memory (32 * E ints, twice).
 constexpr int kSmallWarps = 32;
 
-__global__ void __launch_bounds__(1024) dispatch_small(const int32_t* __restrict__ idx, int TK,
-                                                       int E, int T, int has_shared,
-                                                       int32_t* __restrict__ counts,
-                                                       int32_t* __restrict__ offsets,
-                                                       int32_t* __restrict__ perm,
-                                                       int32_t* __restrict__ inv, TileSpec ts,
-                                                       WsHeader* __restrict__ hdr) {
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ int dyn_smem[];
+// The whole dispatch of at most kChunk copies by one CTA of 1024 threads
+// (dyn_smem: 2 * kSmallWarps * E ints).
+__device__ void dispatch_block(const int32_t* __restrict__ idx, int TK, int E, int T,
+                               int has_shared, int32_t* __restrict__ counts,
+                               int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+                               int32_t* __restrict__ inv, const TileSpec& ts,
+                               WsHeader* __restrict__ hdr, int* dyn_smem) {
   int* cnt = dyn_smem;                      // [kSmallWarps][E]
   int* pre = dyn_smem + kSmallWarps * E;    // [kSmallWarps][E]
   __shared__ int sh[96];
@@ -390,6 +395,19 @@ __global__ void __launch_bounds__(1024) dispatch_small(const int32_t* __restrict
   }
 }
 
+__global__ void __launch_bounds__(1024) dispatch_small(const int32_t* __restrict__ idx, int TK,
+                                                       int E, int T, int has_shared,
+                                                       int32_t* __restrict__ counts,
+                                                       int32_t* __restrict__ offsets,
+                                                       int32_t* __restrict__ perm,
+                                                       int32_t* __restrict__ inv, TileSpec ts,
+                                                       WsHeader* __restrict__ hdr) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int dyn_smem[];
+  dispatch_block(idx, TK, E, T, has_shared, counts, offsets, perm, inv, ts, hdr, dyn_smem);
+}
+
 // Gather of dispatched activation rows: xp[row] = x[perm[row] / K] (bf16,
 // 16-byte vectors), so the tensor-core GEMM reads contiguous rows.
 __global__ void __launch_bounds__(256) gather_rows(const uint4* __restrict__ x,
@@ -426,6 +444,8 @@ static TileSpec make_tile_spec(const moe_layer_desc& d, const WsLayout& L, char*
   ts.m_tiles1_routed = d.D / ts.mtile;
   ts.m_tiles1_shared = d.Ds / ts.mtile;
   ts.m_tiles2 = d.H / ts.mtile;
+  ts.splits1_routed = split ? L.sp.gemm1_routed : 1;
+  ts.splits1_shared = split ? L.sp.gemm1_shared : 1;
   ts.splits2_routed = split ? L.sp.gemm2_routed : 1;
   ts.splits2_shared = split ? L.sp.gemm2_shared : 1;
   return ts;

@@ -41,7 +41,6 @@ constexpr int kStageArea = 192 * 1024;          // shared memory of the operand 
 constexpr int kAccCols = 256;                   // fp32 columns per accumulator
 constexpr int kTmemCols = 2 * kAccCols;
 constexpr int kEpiWarps = 8;                    // two per TMEM lane quarter
-constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr size_t kSmemBytes = 1024 /*barriers*/ + 1024 /*alignment*/ + kStageArea;
@@ -245,6 +244,9 @@ struct Side {          // routed experts (0) or the shared expert (1)
   int m_valid;         // output columns below this bound are stored
   int out_f32;         // 1: fp32 output, 0: bf16 output
   int a_rows;          // rows of the weight box (kBM, or fewer for a short gate matrix)
+  int splits;          // reduction splits of this side's tiles
+  void* fix_out;       // first layer with splits: bf16 GeLU output (out holds fp32 partials)
+  int fix_ld;
 };
 
 struct Args {
@@ -259,6 +261,7 @@ struct Args {
   uint32_t* status;
   int E;
   int gelu;
+  int lockstep;        // 1: some tiles need the split fixup (epilogue warps in lockstep)
 };
 
 // Tile t of the launch: from the list, or (dense tiling, used by the gate
@@ -319,6 +322,62 @@ __device__ __forceinline__ void epilogue_columns(uint32_t taddr, int half, int n
   }
 }
 
+__device__ __forceinline__ void epilogue_bar_sync() {   // the kEpiWarps epilogue warps only
+  asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory");
+}
+
+// First-layer tile with reduction splits, after this CTA stored its fp32
+// partial: the last of the tile's splits to arrive adds the partials of all
+// splits in split order, applies the GeLU and stores the bf16 output. Thread
+// = output column `col`; the two warps of a lane quarter take alternate rows.
+// Arrivals are counted in the split-0 tile of the list (one counter per CTA
+// of a pair), which the dispatch step writes as 0 every forward. All
+// epilogue warps call this together (it holds named barriers).
+constexpr int kFixRows = 4;   // rows per thread and round of loads
+
+__device__ __noinline__ void split_fixup(const Args& args, const Tile& tl, const Side& S,
+                                            uint32_t rank, int half, int col, int n,
+                                            volatile int* owner) {
+  __threadfence();   // this thread's partial stores are visible to the other CTAs
+  epilogue_bar_sync();
+  if (threadIdx.x == 0) {
+    int* arrivals = const_cast<int*>(&args.tiles[tl.first_split].arrivals[rank]);
+    *owner = (atomicAdd(arrivals, 1) == S.splits - 1) ? 1 : 0;
+  }
+  epilogue_bar_sync();
+  if (!*owner) return;
+  __threadfence();   // the other splits' partials are visible to this CTA
+  const float* src = static_cast<const float*>(S.out) + (size_t)tl.r0 * S.ld + col;
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(S.fix_out) + (size_t)tl.r0 * S.fix_ld + col;
+  for (int j0 = half; j0 < n; j0 += 2 * kFixRows) {
+    float a[kFixRows];
+#pragma unroll
+    for (int i = 0; i < kFixRows; ++i) a[i] = 0.f;
+    for (int p0 = 0; p0 < S.splits; p0 += 4) {
+      float v[kFixRows][4];
+#pragma unroll
+      for (int i = 0; i < kFixRows; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int j = j0 + 2 * i;
+          v[i][q] = (j < n && p0 + q < S.splits)
+                        ? __ldcg(src + (size_t)(p0 + q) * S.split_stride + (size_t)j * S.ld)
+                        : 0.f;
+        }
+#pragma unroll
+      for (int i = 0; i < kFixRows; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (p0 + q < S.splits) a[i] = (p0 + q == 0) ? v[i][q] : __fadd_rn(a[i], v[i][q]);
+    }
+#pragma unroll
+    for (int i = 0; i < kFixRows; ++i) {
+      const int j = j0 + 2 * i;
+      if (j < n) dst[(size_t)j * S.fix_ld] = __float2bfloat16_rn(gelu_erf(a[i]));
+    }
+  }
+}
+
 // kPair = false: one CTA per tile of 128 weight rows (MMA M = 128).
 // kPair = true: a cluster of two CTAs per tile of 256 weight rows (one MMA of
 // M = 256 issued by the even CTA); each CTA loads its 128 weight rows and half
@@ -341,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = bars + 2 * kMaxStages + 4;            // [1] all MMAs retired
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMaxStages + 5);
   volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile int* epi_flags = reinterpret_cast<volatile int*>(tmem_slot + 2);   // [4]
   uint8_t* ring = base + 1024;                            // stage s at s * stage_bytes
   const int n_stages = args.n_stages;
   const int stage_bytes = args.stage_bytes;
@@ -519,18 +579,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp w reads TMEM lanes 32*(w%4) .. +31 (thread = weight row of the
     // tile) and every other column chunk of the accumulator, starting at
     // chunk w/4 (column = activation row of the tile).
+    // A launch with split first-layer tiles runs the epilogue warps in
+    // lockstep: one thread waits for each accumulator and the others follow
+    // it through a named barrier, so all of them take the same path through
+    // the barriers of the split fixup. Flags alternate by tile parity: a slot
+    // is rewritten only after every warp has passed the next tile's barrier.
+    // Other launches let each warp wait for the accumulator on its own.
     int acc = 0;
     uint32_t acc_phase = 0;
     const int quarter = warp & 3, half = warp >> 2;
     const int row = (int)rank * kBM + quarter * 32 + lane;
-    for (int t = unit; t < n_tiles; t += n_units) {
+    int it = 0;
+    for (int t = unit; t < n_tiles; t += n_units, ++it) {
       const Tile tl = tile_at(args, t);
       const int sd = (tl.g < args.E) ? 0 : 1;
       const Side& S = args.side[sd];
       int ok = 1;
-      if (lane == 0)
-        ok = wait_bounded(smem_u32(&tfull[acc]), acc_phase, abort_flag, args.status) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (args.lockstep) {
+        if (threadIdx.x == 0)
+          epi_flags[it & 1] =
+              wait_bounded(smem_u32(&tfull[acc]), acc_phase, abort_flag, args.status) ? 1 : 0;
+        epilogue_bar_sync();
+        ok = epi_flags[it & 1];
+      } else {
+        if (lane == 0)
+          ok = wait_bounded(smem_u32(&tfull[acc]), acc_phase, abort_flag, args.status) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
       if (!ok) break;
       tc_fence_after();
       const uint32_t taddr =
@@ -540,7 +615,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t part = (size_t)tl.ks * (size_t)S.split_stride;
       const int n = min(tl.n, n_max);
       const size_t o0 = part + (size_t)tl.r0 * (size_t)S.ld + (size_t)col;
-      if (args.gelu)
+      const bool fix = args.gelu && S.splits > 1;   // split first layer: partial, GeLU later
+      if (fix)
+        epilogue_columns<kEpiF32, 64>(taddr, half, n, store, S.out, o0, S.ld);
+      else if (args.gelu)
         epilogue_columns<kEpiGeluBf16, 32>(taddr, half, n, store, S.out, o0, S.ld);
       else if (S.out_f32)
         epilogue_columns<kEpiF32, 64>(taddr, half, n, store, S.out, o0, S.ld);
@@ -555,6 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           mbar_arrive(te);
       }
+      if (fix) split_fixup(args, tl, S, rank, half, col, n, epi_flags + 2 + (it & 1));
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -656,6 +735,9 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
     s.m_rows = p.m_rows;
     s.m_valid = p.m_valid > 0 ? p.m_valid : p.m_rows;
     s.out_f32 = p.out_f32 ? 1 : 0;
+    s.splits = splits;
+    s.fix_out = p.fix_out;
+    s.fix_ld = p.fix_ld;
     return s;
   };
   Args args;
@@ -680,6 +762,7 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
   args.status = status;
   args.E = E;
   args.gelu = gelu ? 1 : 0;
+  args.lockstep = (gelu && (args.side[0].splits > 1 || args.side[1].splits > 1)) ? 1 : 0;
   if (!pair) {
     const int grid = dense ? std::min(num_sms, std::max(1, dense->tiles)) : num_sms;
     return launch_pdl(grouped_gemm_tc<false>, dim3(grid), dim3(kThreads), kSmemBytes, st, a0, b0,

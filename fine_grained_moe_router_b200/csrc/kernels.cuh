@@ -33,6 +33,10 @@ struct TcProblem {
   int splits;              // reduction splits (0 or 1: none); split s writes out + s * split_stride
   long long split_stride;
   int m_valid;             // output columns stored (0: all m_rows)
+  // First (GeLU) layer with splits > 1: out receives the fp32 partials and
+  // the last split of each tile writes GeLU(sum) as bf16 to fix_out [*, fix_ld].
+  void* fix_out;
+  int fix_ld;
 };
 
 // Tiling without a device tile list (gate GEMM): `rows` activation rows in

@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "kernels.cuh"
 #include "launch.cuh"
+#include "select.cuh"
 
 namespace moe {
 
@@ -89,14 +90,9 @@ __global__ void __launch_bounds__(256) gate_logits_simt(const TIn* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------
-// Top-K selection: one warp per token, lane j holds experts j, j+32, ...
-// K rounds of a warp arg-max by shuffles; the order is (score descending,
-// expert index ascending), so ties go to the lower index and -0.0 == +0.0.
+// Top-K selection kernel: one warp per token (the selection itself is in
+// select.cuh).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ bool better(float sa, int ea, float sb, int eb) {
-  return sa > sb || (sa == sb && ea < eb);
-}
-
 // lrow: the token's logits, given as n_parts partial sums part_stride apart
 // (reduction splits of the gate GEMM), added in split order; the total is
 // written to logits_out when it is non-null.
@@ -144,44 +140,7 @@ __device__ __forceinline__ void select_row(const float* __restrict__ lrow, int n
       s[j] = -INFINITY;
     }
   }
-  uint32_t taken = 0;
-  float my_s = -INFINITY;   // score of slot `lane` (lane < K)
-  int my_e = 0;
-  for (int k = 0; k < K; ++k) {
-    float bs = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E && !((taken >> j) & 1u) && better(s[j], e, bs, be)) {
-        bs = s[j];
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (better(os, oe, bs, be)) {
-        bs = os;
-        be = oe;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == k) {
-      my_s = bs;
-      my_e = be;
-    }
-  }
-  // w_k = exp(s_k - s_0) / sum_{j<K} exp(s_j - s_0), summed in slot order.
-  const float s0 = __shfl_sync(0xffffffffu, my_s, 0);
-  const float z = (lane < K) ? expf(my_s - s0) : 0.f;
-  float den = 0.f;
-  for (int j = 0; j < K; ++j) den += __shfl_sync(0xffffffffu, z, j);
-  if (lane < K) {
-    idx_out[lane] = my_e;
-    w_out[lane] = z / den;
-  }
+  select_topk_warp<NJ>(s, E, K, idx_out, w_out);
 }
 
 template <int NJ>
