@@ -96,6 +96,16 @@ def draw_x(wl: Workload, T: int, replica: int = 0) -> torch.Tensor:
     return _normal((T, wl.H), 1.0, g, torch_dtype(wl))
 
 
+def draw_gumbel(T: int, E: int, seed: int) -> torch.Tensor:
+    """Standard Gumbel draws g [T, E] fp32, g = -log(-log(u)) with u uniform in
+    (0, 1): the random input of noisy routing, drawn here so that the oracle
+    and the GPU path see the same numbers."""
+    g = _gen(seed * 7 + 3)
+    u = torch.rand((T, E), generator=g, dtype=torch.float64)
+    u = u.clamp(min=1e-12, max=1.0 - 1e-12)
+    return (-torch.log(-torch.log(u))).to(torch.float32)
+
+
 def draw_router(wl: Workload) -> torch.Tensor:
     """Gate weight W_r [E, H] ~ N(0, 1/H) (nn.Linear(H, E, bias=False) layout)."""
     return _normal((wl.E, wl.H), 1.0 / math.sqrt(wl.H), _gen(_base(wl) + 1), torch_dtype(wl))

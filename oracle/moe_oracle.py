@@ -65,7 +65,7 @@ def router_logits(x: np.ndarray, w_router: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------
 # a2  bias + top-K selection + renormalisation
 # --------------------------------------------------------------------------
-def selection_scores(logits: np.ndarray, bias) -> np.ndarray:
+def selection_scores(logits: np.ndarray, bias, noise=None) -> np.ndarray:
     """The fp32 scores the selection is decided on: ``s = fl32(fl32(l) + B)``.
 
     [K3-DIAG] 四: the expert bias B is added to the logits before the
@@ -73,14 +73,23 @@ def selection_scores(logits: np.ndarray, bias) -> np.ndarray:
     kernel's precision): softmax is strictly increasing, so in exact
     arithmetic it selects the same set, and deciding on fp32 ``l + B`` avoids
     ties created or merged by rounding of exp.
+
+    [MOE-ARCH] §2.3 (inference): Gumbel noise is added to the logits before
+    the softmax, so the top-K choice is randomised and hot experts do not
+    stay fixed. ``noise`` is a [T, E] array of Gumbel(0, 1) draws supplied by
+    the caller; the scores are then ``fl32(fl32(l + B) + g)`` and the weights
+    come from the softmax of these noisy scores.
     """
     l32 = np.asarray(logits, dtype=np.float64).astype(np.float32)
     E = l32.shape[-1]
     b32 = np.zeros(E, np.float32) if bias is None else np.asarray(bias, dtype=np.float32)
-    return (l32 + b32[None, :]).astype(np.float32)
+    s = (l32 + b32[None, :]).astype(np.float32)
+    if noise is not None:
+        s = (s + np.asarray(noise, dtype=np.float32)).astype(np.float32)
+    return s
 
 
-def select_topk(logits: np.ndarray, bias, K: int):
+def select_topk(logits: np.ndarray, bias, K: int, noise=None):
     """Top-K experts per token and their renormalised weights.
 
     [K3-A2A] "工业级细粒度 MoE 路由与通信掩盖实战": scores = softmax(logits),
@@ -92,7 +101,7 @@ def select_topk(logits: np.ndarray, bias, K: int):
     The weights are ``exp(s_k - s_max) / sum_{j in sel} exp(s_j - s_max)``:
     the full-E softmax denominator cancels in the renormalisation.
     """
-    s = selection_scores(logits, bias)
+    s = selection_scores(logits, bias, noise)
     T, E = s.shape
     if not 1 <= K <= E:
         raise ValueError("need 1 <= K <= E")
@@ -227,7 +236,7 @@ def combine(y_rows, w, inv, y_shared=None):
 # --------------------------------------------------------------------------
 # a9  full layer: route, dispatch, experts, weighted combine (+ shared)
 # --------------------------------------------------------------------------
-def moe_layer_forward(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None):
+def moe_layer_forward(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None, noise=None):
     """Forward pass of one fine-grained MoE FFN layer.
 
     Steps: gate logits, Softmax(l + B) selection of the top K with
@@ -242,6 +251,8 @@ def moe_layer_forward(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None):
     ``w1``/``w2`` only need ``w1[e]`` indexing (lazy widening is allowed).
     ``tokens``: optional sorted token indices; the output is computed for
     those tokens only (routing and dispatch always cover all T tokens).
+    ``noise``: optional [T, E] Gumbel draws for noisy routing ([MOE-ARCH]
+    §2.3; see ``selection_scores``).
 
     Returns dict with logits, idx, w, s, counts, offsets, perm, inv and
     ``y`` [len(tokens), H] float64.
@@ -250,7 +261,7 @@ def moe_layer_forward(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None):
     T, H = x.shape
     E = np.asarray(w_router).shape[0]
     logits = router_logits(x, w_router)
-    idx, w, s = select_topk(logits, bias, K)
+    idx, w, s = select_topk(logits, bias, K, noise)
     counts, off, perm, inv = dispatch(idx, E)
 
     tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)

@@ -19,8 +19,8 @@ _orig = {n: getattr(om, n) for n in ("select_topk", "dispatch", "gelu_erf", "gin
                                       "moe_layer_forward")}
 
 
-def _topk_high_index_ties(logits, bias, K):
-    s = om.selection_scores(logits, bias)
+def _topk_high_index_ties(logits, bias, K, noise=None):
+    s = om.selection_scores(logits, bias, noise)
     order = np.argsort(-s.astype(np.float64)[:, ::-1], axis=1, kind="stable")
     idx = (s.shape[1] - 1 - order[:, :K]).astype(np.int32)
     ss = np.take_along_axis(s, idx, 1).astype(np.float64)
@@ -28,21 +28,34 @@ def _topk_high_index_ties(logits, bias, K):
     return idx, z / z.sum(1, keepdims=True), s
 
 
-def _topk_no_renorm(logits, bias, K):
-    idx, _, s = _orig["select_topk"](logits, bias, K)
+def _topk_no_renorm(logits, bias, K, noise=None):
+    idx, _, s = _orig["select_topk"](logits, bias, K, noise)
     s64 = s.astype(np.float64)
     p = np.exp(s64 - s64.max(1, keepdims=True))
     p /= p.sum(1, keepdims=True)
     return idx, np.take_along_axis(p, idx, 1), s
 
 
-def _scores_ignore_bias(logits, bias):
-    return _orig["selection_scores"](logits, None)
+def _scores_ignore_bias(logits, bias, noise=None):
+    return _orig["selection_scores"](logits, None, noise)
 
 
-def _scores_fp64(logits, bias):
+def _scores_fp64(logits, bias, noise=None):
     b = 0.0 if bias is None else np.asarray(bias, np.float64)[None, :]
-    return np.asarray(logits, np.float64) + b
+    g = 0.0 if noise is None else np.asarray(noise, np.float64)
+    return np.asarray(logits, np.float64) + b + g
+
+
+def _scores_ignore_noise(logits, bias, noise=None):
+    return _orig["selection_scores"](logits, bias, None)
+
+
+def _topk_weights_from_clean_scores(logits, bias, K, noise=None):
+    idx, _, s = _orig["select_topk"](logits, bias, K, noise)
+    clean = _orig["selection_scores"](logits, bias, None).astype(np.float64)
+    sel = np.take_along_axis(clean, idx, 1)
+    z = np.exp(sel - sel.max(1, keepdims=True))
+    return idx, z / z.sum(1, keepdims=True), s
 
 
 def _dispatch_descending(idx, E):
@@ -89,8 +102,8 @@ def _ffn_transposed_second(rows, w1, w2):
     return h @ w2.T * 1.0001
 
 
-def _layer_no_shared(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None):
-    return _orig["moe_layer_forward"](x, w_router, bias, w1, w2, None, None, K, tokens)
+def _layer_no_shared(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None, noise=None):
+    return _orig["moe_layer_forward"](x, w_router, bias, w1, w2, None, None, K, tokens, noise)
 
 
 def _stats_overflow_counts_experts(counts, T, K, cf_num=5, cf_den=4):
@@ -113,6 +126,8 @@ MUTANTS = {
     "ffn_second_linear_transposed": ("expert_ffn", _ffn_transposed_second),
     "shared_expert_dropped": ("moe_layer_forward", _layer_no_shared),
     "overflow_counts_experts": ("load_stats", _stats_overflow_counts_experts),
+    "gumbel_noise_ignored": ("selection_scores", _scores_ignore_noise),
+    "noisy_weights_from_clean_scores": ("select_topk", _topk_weights_from_clean_scores),
 }
 
 PIN_TESTS = [
@@ -132,6 +147,8 @@ PIN_TESTS = [
     pins.test_gini_matches_mean_absolute_difference_form,
     pins.test_load_stats_golden_cases,
     pins.test_capacity_integer_form_equals_page_float_form,
+    pins.test_gumbel_max_picks_each_expert_with_its_softmax_probability,
+    pins.test_noisy_weights_are_the_softmax_of_the_noisy_scores,
 ]
 
 

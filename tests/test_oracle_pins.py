@@ -408,3 +408,69 @@ def test_repeated_bias_updates_even_out_a_skewed_router():
         b = oracle.bias_update(b, counts, T, K, 0.02)
     g1 = oracle.gini_exact(oracle.expert_counts(oracle.select_topk(logits, b, K)[0], E))
     assert g1 < 0.6 * g0
+
+
+# ------------------------------------------------------ Gumbel-noise routing ---
+def _gumbel(rng, shape):
+    u = rng.uniform(size=shape)
+    return (-np.log(-np.log(u))).astype(np.float32)
+
+
+def test_noisy_routing_without_noise_is_plain_routing():
+    rng = np.random.default_rng(5)
+    l = rng.normal(size=(40, 12))
+    b = rng.uniform(-0.3, 0.3, 12).astype(np.float32)
+    i0, w0, s0 = oracle.select_topk(l, b, 3)
+    i1, w1, s1 = oracle.select_topk(l, b, 3, noise=np.zeros((40, 12), np.float32))
+    assert (i0 == i1).all() and np.array_equal(w0, w1) and np.array_equal(s0, s1)
+
+
+def _softmax(v):
+    z = np.exp(v - v.max())
+    return z / z.sum()
+
+
+def test_gumbel_max_picks_each_expert_with_its_softmax_probability():
+    """Gumbel-max: argmax_e (l_e + B_e + g_e) with standard Gumbel g is e with
+    probability softmax(l + B)_e (the selection probabilities the page's
+    noisy softmax routing gives at K = 1)."""
+    rng = np.random.default_rng(11)
+    E, N = 5, 200_000
+    l = np.array([0.3, -0.4, 1.1, 0.0, -1.5])
+    b = np.array([0.1, 0.2, -0.3, 0.0, 0.25], np.float32)
+    p = _softmax(l + b.astype(np.float64))
+    idx, w, _ = oracle.select_topk(np.tile(l, (N, 1)), b, 1, noise=_gumbel(rng, (N, E)))
+    freq = np.bincount(idx[:, 0], minlength=E) / N
+    assert np.all(np.abs(freq - p) <= 5 * np.sqrt(p * (1 - p) / N))
+    assert np.all(w == 1.0)
+
+
+def test_gumbel_top2_follows_plackett_luce_order():
+    """Gumbel-top-k: the first two slots are experts a then b with
+    probability p_a * p_b / (1 - p_a) (sampling without replacement in
+    proportion to softmax(l + B))."""
+    rng = np.random.default_rng(12)
+    E, N = 4, 200_000
+    l = np.array([0.5, -0.2, 0.9, -1.0])
+    p = _softmax(l)
+    idx, _, _ = oracle.select_topk(np.tile(l, (N, 1)), None, 2, noise=_gumbel(rng, (N, E)))
+    pair = idx[:, 0] * E + idx[:, 1]
+    freq = np.bincount(pair, minlength=E * E) / N
+    for a in range(E):
+        for c in range(E):
+            q = 0.0 if a == c else p[a] * p[c] / (1 - p[a])
+            assert abs(freq[a * E + c] - q) <= 5 * math.sqrt(max(q * (1 - q), 1e-12) / N) + 1e-12
+
+
+def test_noisy_weights_are_the_softmax_of_the_noisy_scores():
+    rng = np.random.default_rng(13)
+    l = rng.normal(size=(30, 9))
+    b = rng.uniform(-0.5, 0.5, 9).astype(np.float32)
+    g = _gumbel(rng, (30, 9))
+    idx, w, s = oracle.select_topk(l, b, 4, noise=g)
+    want = ((l.astype(np.float32) + b).astype(np.float32) + g).astype(np.float32)
+    assert np.array_equal(s, want)
+    sel = np.take_along_axis(s.astype(np.float64), idx, 1)
+    assert np.all(np.diff(sel, axis=1) <= 0)                      # slots by descending noisy score
+    np.testing.assert_allclose(w.sum(1), 1.0, atol=1e-12)
+    np.testing.assert_allclose(w[:, 1:] / w[:, :1], np.exp(sel[:, 1:] - sel[:, :1]), rtol=1e-12)
