@@ -21,7 +21,8 @@ MOE_F32, MOE_BF16 = 0, 1
 
 # Every symbol include/moe.h declares.
 EXPORTED = (
-    "moe_workspace_size", "moe_router_topk", "moe_topk_from_logits", "moe_dispatch",
+    "moe_workspace_size", "moe_router_topk", "moe_topk_from_logits", "moe_topk_from_logits_noisy",
+    "moe_dispatch", "moe_layer_forward_noisy",
     "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
     "moe_expert_stats", "moe_bias_update",
     "moe_check_status", "moe_status_string", "moe_kernel_launch_count", "moe_dispatch_noalloc",
@@ -68,6 +69,9 @@ def _load() -> ctypes.CDLL:
         "moe_workspace_size": (S, [D]),
         "moe_router_topk": (ctypes.c_int, [D, P, P, P, P, P, P, P, S, P]),
         "moe_topk_from_logits": (ctypes.c_int, [D, P, P, P, P, P]),
+        "moe_topk_from_logits_noisy": (ctypes.c_int, [D, P, P, P, P, P, P]),
+        "moe_layer_forward_noisy": (ctypes.c_int, [D, ctypes.POINTER(MoELayerWeights), P, P, P,
+                                                   ctypes.POINTER(MoERouting), P, S, P]),
         "moe_dispatch": (ctypes.c_int, [D, P, P, P, P, P, P, S, P]),
         "moe_grouped_ffn": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, S, P]),
         "moe_combine": (ctypes.c_int, [D, P, P, P, P, P, P]),
@@ -148,6 +152,13 @@ def moe_topk_from_logits(desc, logits, bias, topk_idx, topk_w, stream=None):
                                     _p(topk_w), _stream(stream)), "moe_topk_from_logits")
 
 
+def moe_topk_from_logits_noisy(desc, logits, bias, gumbel_noise, topk_idx, topk_w, stream=None):
+    """Selection on (logits + bias) + gumbel_noise [T, E] fp32 (noisy routing)."""
+    _check(lib.moe_topk_from_logits_noisy(ctypes.byref(desc), _p(logits), _p(bias),
+                                          _p(gumbel_noise), _p(topk_idx), _p(topk_w),
+                                          _stream(stream)), "moe_topk_from_logits_noisy")
+
+
 def moe_dispatch(desc, topk_idx, counts, offsets, perm, inv, ws, stream=None):
     _check(lib.moe_dispatch(ctypes.byref(desc), _p(topk_idx), _p(counts), _p(offsets), _p(perm),
                             _p(inv), _p(ws), ws.numel() if ws is not None else 0, _stream(stream)),
@@ -191,6 +202,16 @@ def moe_layer_forward(desc, weights: MoELayerWeights, x, y, routing: Optional[Mo
                                  ctypes.byref(routing) if routing is not None else None, _p(ws),
                                  ws.numel() if ws is not None else 0, _stream(stream)),
            "moe_layer_forward")
+
+
+def moe_layer_forward_noisy(desc, weights: MoELayerWeights, x, gumbel_noise, y,
+                            routing: Optional[MoERouting], ws, stream=None):
+    """moe_layer_forward with Gumbel noise [T, E] fp32 added to the selection scores."""
+    _check(lib.moe_layer_forward_noisy(ctypes.byref(desc), ctypes.byref(weights), _p(x),
+                                       _p(gumbel_noise), _p(y),
+                                       ctypes.byref(routing) if routing is not None else None,
+                                       _p(ws), ws.numel() if ws is not None else 0,
+                                       _stream(stream)), "moe_layer_forward_noisy")
 
 
 FORWARD_STAGES = ("router", "dispatch", "gemm1", "gemm2", "combine")

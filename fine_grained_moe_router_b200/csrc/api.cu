@@ -352,17 +352,18 @@ static moe_status run_grouped_ffn(const moe_layer_desc& d, const WsLayout& L, ch
 // kernel); fp32 layers on CUDA cores.
 static moe_status run_router(const moe_layer_desc& d, const WsLayout& L, char* ws,
                              const void* x, const void* wr, const float* bias, int32_t* idx,
-                             float* tw, float* logits_out, cudaStream_t st) {
+                             float* tw, float* logits_out, cudaStream_t st,
+                             const float* noise = nullptr) {
   if (d.T == 0) return MOE_OK;
   if (d.dtype == MOE_BF16) {
     float* parts = reinterpret_cast<float*>(ws + L.logits_part);
     MOE_CUDA_TRY(launch_gate_logits_tc(d, L, ws, x, wr, parts, num_sms(), st));
-    MOE_CUDA_TRY(launch_topk_select(d, parts, L.sp.router, (size_t)d.T * d.E, bias, idx, tw,
-                                    logits_out, st));
+    MOE_CUDA_TRY(launch_topk_select(d, parts, L.sp.router, (size_t)d.T * d.E, bias, noise, idx,
+                                    tw, logits_out, st));
   } else {
     float* logits = logits_out ? logits_out : reinterpret_cast<float*>(ws + L.logits);
     MOE_CUDA_TRY(launch_gate_logits(d, x, wr, logits, st));
-    MOE_CUDA_TRY(launch_topk_select(d, logits, 1, 0, bias, idx, tw, nullptr, st));
+    MOE_CUDA_TRY(launch_topk_select(d, logits, 1, 0, bias, noise, idx, tw, nullptr, st));
   }
   return MOE_OK;
 }
@@ -394,17 +395,30 @@ moe_status moe_router_topk(const moe_layer_desc* desc, const void* x, const void
                     logits_or_null, st);
 }
 
-moe_status moe_topk_from_logits(const moe_layer_desc* desc, const float* logits,
-                                const float* bias, int32_t* topk_idx, float* topk_w,
-                                moe_stream stream) {
+static moe_status topk_from_logits_impl(const moe_layer_desc* desc, const float* logits,
+                                        const float* bias, const float* noise, int32_t* topk_idx,
+                                        float* topk_w, moe_stream stream) {
   MOE_TRY(check_desc(desc));
   const moe_layer_desc& d = *desc;
   if (d.T == 0) return MOE_OK;
   MOE_TRY(check_ptrs({logits, topk_idx, topk_w}));
   if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
-  MOE_CUDA_TRY(launch_topk_select(d, logits, 1, 0, bias, topk_idx, topk_w, nullptr,
+  MOE_CUDA_TRY(launch_topk_select(d, logits, 1, 0, bias, noise, topk_idx, topk_w, nullptr,
                                   static_cast<cudaStream_t>(stream)));
   return MOE_OK;
+}
+
+moe_status moe_topk_from_logits(const moe_layer_desc* desc, const float* logits,
+                                const float* bias, int32_t* topk_idx, float* topk_w,
+                                moe_stream stream) {
+  return topk_from_logits_impl(desc, logits, bias, nullptr, topk_idx, topk_w, stream);
+}
+
+moe_status moe_topk_from_logits_noisy(const moe_layer_desc* desc, const float* logits,
+                                      const float* bias, const float* gumbel_noise,
+                                      int32_t* topk_idx, float* topk_w, moe_stream stream) {
+  if (!gumbel_noise || !aligned16(gumbel_noise)) return MOE_ERR_INVALID_ARG;
+  return topk_from_logits_impl(desc, logits, bias, gumbel_noise, topk_idx, topk_w, stream);
 }
 
 moe_status moe_dispatch(const moe_layer_desc* desc, const int32_t* topk_idx, int32_t* counts,
@@ -457,7 +471,8 @@ moe_status moe_combine(const moe_layer_desc* desc, const void* y_rows, const flo
 static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer_weights* weights,
                                      const void* x, void* y, const moe_routing* routing_or_null,
                                      void* ws, size_t ws_bytes, cudaStream_t st,
-                                     cudaEvent_t const* ev, int n_ev) {
+                                     cudaEvent_t const* ev, int n_ev,
+                                     const float* noise = nullptr) {
   MOE_TRY(check_desc(desc));
   const moe_layer_desc& d = *desc;
   MOE_TRY(check_ws(d, ws, ws_bytes));
@@ -487,7 +502,7 @@ static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer
   auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
 
   MOE_CUDA_TRY(mark(0));
-  MOE_TRY(run_router(d, L, w, x, W.w_router, W.expert_bias, idx, tw, R.logits, st));
+  MOE_TRY(run_router(d, L, w, x, W.w_router, W.expert_bias, idx, tw, R.logits, st, noise));
   MOE_CUDA_TRY(mark(1));
   const bool tc = d.dtype == MOE_BF16;
   MOE_CUDA_TRY(launch_dispatch(d, L, w, idx, counts, offsets, perm, inv, tc, st));
@@ -506,6 +521,15 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights
                              void* ws, size_t ws_bytes, moe_stream stream) {
   return layer_forward_impl(desc, weights, x, y, routing_or_null, ws, ws_bytes,
                             static_cast<cudaStream_t>(stream), nullptr, 0);
+}
+
+moe_status moe_layer_forward_noisy(const moe_layer_desc* desc, const moe_layer_weights* weights,
+                                   const void* x, const float* gumbel_noise, void* y,
+                                   const moe_routing* routing_or_null, void* ws, size_t ws_bytes,
+                                   moe_stream stream) {
+  if (!gumbel_noise || !aligned16(gumbel_noise)) return MOE_ERR_INVALID_ARG;
+  return layer_forward_impl(desc, weights, x, y, routing_or_null, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream), nullptr, 0, gumbel_noise);
 }
 
 moe_status moe_layer_forward_profiled(const moe_layer_desc* desc,

@@ -54,9 +54,10 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
 
 cudaError_t launch_gate_logits(const moe_layer_desc& d, const void* x, const void* wr,
                                float* logits, cudaStream_t st);
+// noise (nullable): Gumbel draws [T, E] fp32 added after the bias.
 cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, int n_parts,
-                               size_t part_stride, const float* bias, int32_t* idx, float* w,
-                               float* logits_out, cudaStream_t st);
+                               size_t part_stride, const float* bias, const float* noise,
+                               int32_t* idx, float* w, float* logits_out, cudaStream_t st);
 // Gate logits on the tensor cores (bf16 layers): `parts` receives
 // L.sp.router partial sums [T, E] fp32, part stride T * E.
 cudaError_t launch_gate_logits_tc(const moe_layer_desc& d, const WsLayout& L, char* ws,

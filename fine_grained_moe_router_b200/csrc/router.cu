@@ -95,11 +95,14 @@ __global__ void __launch_bounds__(256) gate_logits_simt(const TIn* __restrict__ 
 // ---------------------------------------------------------------------------
 // lrow: the token's logits, given as n_parts partial sums part_stride apart
 // (reduction splits of the gate GEMM), added in split order; the total is
-// written to logits_out when it is non-null.
+// written to logits_out when it is non-null. grow (nullable): the token's
+// Gumbel noise for noisy routing ("MoE architecture in production" §2.3),
+// added in fp32 after the bias: s = (l + B) + g.
 template <int NJ>
 __device__ __forceinline__ void select_row(const float* __restrict__ lrow, int n_parts,
                                            size_t part_stride, const float* __restrict__ bias,
-                                           int E, int K, int32_t* __restrict__ idx_out,
+                                           const float* __restrict__ grow, int E, int K,
+                                           int32_t* __restrict__ idx_out,
                                            float* __restrict__ w_out,
                                            float* __restrict__ logits_out) {
   const int lane = threadIdx.x & 31;
@@ -136,6 +139,7 @@ __device__ __forceinline__ void select_row(const float* __restrict__ lrow, int n
       if (logits_out) logits_out[e] = l[j];
       const float b = bias ? bias[e] : 0.f;
       s[j] = __fadd_rn(l[j], b);
+      if (grow) s[j] = __fadd_rn(s[j], grow[e]);   // Gumbel noise, after the bias
     } else {
       s[j] = -INFINITY;
     }
@@ -146,7 +150,8 @@ __device__ __forceinline__ void select_row(const float* __restrict__ lrow, int n
 template <int NJ>
 __global__ void __launch_bounds__(256) topk_select_kernel(const float* __restrict__ logits,
                                                           int n_parts, size_t part_stride,
-                                                          const float* __restrict__ bias, int T,
+                                                          const float* __restrict__ bias,
+                                                          const float* __restrict__ noise, int T,
                                                           int E, int K,
                                                           int32_t* __restrict__ idx,
                                                           float* __restrict__ w,
@@ -155,7 +160,8 @@ __global__ void __launch_bounds__(256) topk_select_kernel(const float* __restric
   pdl_trigger();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
-  select_row<NJ>(logits + (size_t)t * E, n_parts, part_stride, bias, E, K, idx + (size_t)t * K,
+  select_row<NJ>(logits + (size_t)t * E, n_parts, part_stride, bias,
+                 noise ? noise + (size_t)t * E : nullptr, E, K, idx + (size_t)t * K,
                  w + (size_t)t * K, logits_out ? logits_out + (size_t)t * E : nullptr);
 }
 
@@ -205,15 +211,15 @@ cudaError_t launch_gate_logits_tc(const moe_layer_desc& d, const WsLayout& L, ch
 }
 
 cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, int n_parts,
-                               size_t part_stride, const float* bias, int32_t* idx, float* w,
-                               float* logits_out, cudaStream_t st) {
+                               size_t part_stride, const float* bias, const float* noise,
+                               int32_t* idx, float* w, float* logits_out, cudaStream_t st) {
   if (d.T == 0) return cudaSuccess;
   const int nj = (d.E + 31) / 32;
   dim3 grid((d.T + 7) / 8);
 #define MOE_TOPK_CASE(NJ)                                                                    \
   case NJ:                                                                                   \
     return launch_pdl(topk_select_kernel<NJ>, grid, dim3(256), 0, st, logits, n_parts,       \
-                      part_stride, bias, d.T, d.E, d.K, idx, w, logits_out);
+                      part_stride, bias, noise, d.T, d.E, d.K, idx, w, logits_out);
   switch (nj) {
     MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4)
     MOE_TOPK_CASE(5) MOE_TOPK_CASE(6) MOE_TOPK_CASE(7) MOE_TOPK_CASE(8)

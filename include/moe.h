@@ -144,6 +144,19 @@ moe_status moe_topk_from_logits(const moe_layer_desc* desc, const float* logits,
                                 const float* bias, int32_t* topk_idx, float* topk_w,
                                 moe_stream stream);
 
+/* Noisy routing: "MoE architecture in production" §2.3 adds Gumbel noise to
+ * the logits before the softmax at inference, so the top-K choice is
+ * randomised and hot experts do not stay fixed. The caller draws the noise:
+ *   gumbel_noise [T, E] fp32 (device, required, 16-byte aligned), standard
+ *   Gumbel draws (e.g. -log(-log(u)), u uniform in (0, 1)); scaling them
+ *   sets the temperature.
+ * Scores s = (l + B) + g, each add in fp32 in that order; selection, slot
+ * order and weights (renormalised softmax of the selected noisy scores) as
+ * in moe_topk_from_logits. Deterministic for given noise. */
+moe_status moe_topk_from_logits_noisy(const moe_layer_desc* desc, const float* logits,
+                                      const float* bias, const float* gumbel_noise,
+                                      int32_t* topk_idx, float* topk_w, moe_stream stream);
+
 /* Dispatch: per-expert histogram, exclusive prefix-sum offsets and the
  * stable permutation of the T*K copies into expert-contiguous rows.
  * "MoE architecture in production" §3.1 (MoEDispatcher.dispatch);
@@ -207,6 +220,16 @@ moe_status moe_combine(const moe_layer_desc* desc, const void* y_rows, const flo
 moe_status moe_layer_forward(const moe_layer_desc* desc, const moe_layer_weights* weights,
                              const void* x, void* y, const moe_routing* routing_or_null,
                              void* ws, size_t ws_bytes, moe_stream stream);
+
+/* moe_layer_forward with noisy routing (see moe_topk_from_logits_noisy):
+ * gumbel_noise [T, E] fp32 (device, required) is added to l + B before the
+ * top-K; everything after the selection is unchanged. Graph capture as for
+ * moe_layer_forward (the noise pointer is captured; refill its contents
+ * before each replay). */
+moe_status moe_layer_forward_noisy(const moe_layer_desc* desc, const moe_layer_weights* weights,
+                                   const void* x, const float* gumbel_noise, void* y,
+                                   const moe_routing* routing_or_null, void* ws, size_t ws_bytes,
+                                   moe_stream stream);
 
 /* moe_layer_forward that also records caller-created CUDA events
  * (cudaEvent_t passed as plain pointers, n_events >= 6) on `stream`

@@ -39,9 +39,10 @@ def rel_max_err(got: np.ndarray, ref: np.ndarray) -> float:
     return float(np.max(np.abs(got - ref))) / max(rms, 1e-30)
 
 
-def scores64(logits64: np.ndarray, bias) -> np.ndarray:
+def scores64(logits64: np.ndarray, bias, noise=None) -> np.ndarray:
     b = np.zeros(logits64.shape[1]) if bias is None else np.asarray(bias, np.float64)
-    return logits64 + b[None, :]
+    s = logits64 + b[None, :]
+    return s if noise is None else s + np.asarray(noise, np.float64)
 
 
 def unique_selection_mask(s64: np.ndarray, K: int, tol: float) -> np.ndarray:
@@ -69,17 +70,17 @@ def check_selection_valid(idx: np.ndarray, s64: np.ndarray, tol: float):
         assert (np.diff(chosen) <= 2 * tol).all()
 
 
-def compare_routing(wl, gpu_logits, gpu_idx, gpu_w, ref_logits64, bias):
+def compare_routing(wl, gpu_logits, gpu_idx, gpu_w, ref_logits64, bias, noise=None):
     """Returns (unique mask, oracle routing) after checking logits, selection
     and weights as described in the module doc."""
     K = wl.K
     rms = float(np.sqrt(np.mean(ref_logits64 ** 2))) if ref_logits64.size else 1.0
     lerr = float(np.max(np.abs(gpu_logits.astype(np.float64) - ref_logits64))) if ref_logits64.size else 0.0
     assert lerr <= logit_tol(wl) * rms, f"logit error {lerr / rms:.3e} x RMS"
-    s64 = scores64(ref_logits64, bias)
+    s64 = scores64(ref_logits64, bias, noise)
     tol = lerr + 2.0 ** -22 * (float(np.abs(s64).max()) if s64.size else 0.0)
     uniq = unique_selection_mask(s64, K, tol)
-    ref_idx, ref_w, _ = oracle.select_topk(ref_logits64, bias, K)
+    ref_idx, ref_w, _ = oracle.select_topk(ref_logits64, bias, K, noise)
     assert (gpu_idx[uniq] == ref_idx[uniq]).all(), "selection differs on a token with a unique answer"
     # w_k = softmax of the chosen scores: dw_k/ds_j = w_k (delta_kj - w_j), so a
     # score error e moves each weight by at most 2 e (plus fp32 rounding).

@@ -125,6 +125,11 @@ def test_argument_errors_are_reported_before_any_launch(M):
     assert lib.moe_topk_from_logits(ctypes.byref(bad), ws, None, ws, ws, None) == 1
     uns = M.make_desc(8, 200, 16, 2, 512, 0, M.MOE_BF16)
     assert lib.moe_topk_from_logits(ctypes.byref(uns), ws, None, ws, ws, None) == 2
+    # noisy routing: the noise tensor is required and aligned
+    assert lib.moe_topk_from_logits_noisy(ctypes.byref(d), ws, None, None, ws, ws, None) == 1
+    assert lib.moe_topk_from_logits_noisy(ctypes.byref(d), ws, None, odd, ws, ws, None) == 1
+    assert lib.moe_layer_forward_noisy(ctypes.byref(d), ctypes.byref(w), ws, None, ws, None, ws,
+                                       need, None) == 1
     # bias update: missing buffers, negative or non-finite step
     assert lib.moe_bias_update(ctypes.byref(d), None, ws, 0.1, None) == 1
     assert lib.moe_bias_update(ctypes.byref(d), ws, ws, -0.1, None) == 1
