@@ -453,14 +453,15 @@ static TileSpec make_tile_spec(const moe_layer_desc& d, const WsLayout& L, char*
 
 cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws,
                             const int32_t* idx, int32_t* counts, int32_t* offsets,
-                            int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st) {
+                            int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st,
+                            bool shared_tiles) {
   const int TK = d.T * d.K;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
   int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
   const int n_chunks = L.n_chunks;
   const TileSpec ts = make_tile_spec(d, L, ws, tc_tiles, /*split=*/true);
-  const int has_shared = d.Ds > 0 ? 1 : 0;
+  const int has_shared = (d.Ds > 0 && shared_tiles) ? 1 : 0;
   if (TK > 0 && TK <= kChunk) {
     const size_t smem = sizeof(int) * 2 * kSmallWarps * (size_t)d.E;
     static bool attr_set[64] = {false};   // per device: dynamic smem above 48 KB

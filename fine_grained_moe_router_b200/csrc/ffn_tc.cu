@@ -255,6 +255,7 @@ struct Args {
   const int* n_tiles;  // device tile count of the list
   int dense_tiles;     // dense tiling: row tiles x weight-row tiles x splits
   int dense_rows, dense_m_tiles, dense_splits;
+  int dense_mtile;     // weight rows per dense tile: kBM, or 2 * kBM on CTA pairs
   int nbox_max;        // activation boxes per stage (rows per tile <= 32 * nbox_max)
   int stage_bytes;     // kABytes + nbox_max * kBoxBytes
   int n_stages;        // stages in the ring (<= kMaxStages)
@@ -271,7 +272,7 @@ __device__ __forceinline__ Tile tile_at(const Args& a, int t) {
   Tile tl;
   tl.ks = t % a.dense_splits;
   const int q = t / a.dense_splits;
-  tl.m0 = (q % a.dense_m_tiles) * kBM;
+  tl.m0 = (q % a.dense_m_tiles) * a.dense_mtile;
   tl.r0 = (q / a.dense_m_tiles) * kTcRows;
   tl.n = min(kTcRows, a.dense_rows - tl.r0);
   tl.g = 0;
@@ -694,9 +695,10 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
 cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& shared, int E,
                                    bool gelu, const Tile* tiles, const int* n_tiles,
                                    const DenseTiling* dense, bool pair, uint32_t* status,
-                                   int num_sms, cudaStream_t st) {
+                                   int num_sms, cudaStream_t st, int max_ctas) {
   using namespace tc;
-  if (pair && dense) return cudaErrorInvalidValue;   // the gate GEMM runs single-CTA tiles
+  // a split first layer needs the tile list (its fixup counts arrivals there)
+  if (dense && gelu && routed.splits > 1) return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};   // per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -749,6 +751,7 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
   args.dense_rows = dense ? dense->rows : 0;
   args.dense_m_tiles = dense ? dense->m_tiles : 1;
   args.dense_splits = dense ? (routed.splits > 0 ? routed.splits : 1) : 1;
+  args.dense_mtile = pair ? 2 * kBM : kBM;
   // Ring shape: no tile has more rows than its activation matrix, so small
   // batches get small activation boxes per stage and a deeper ring (more
   // weight bytes in flight per SM). A CTA of a pair loads half of the rows.
@@ -763,12 +766,14 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
   args.E = E;
   args.gelu = gelu ? 1 : 0;
   args.lockstep = (gelu && (args.side[0].splits > 1 || args.side[1].splits > 1)) ? 1 : 0;
+  const int sms = (max_ctas > 0) ? std::min(num_sms, max_ctas) : num_sms;
   if (!pair) {
-    const int grid = dense ? std::min(num_sms, std::max(1, dense->tiles)) : num_sms;
+    const int grid = dense ? std::min(sms, std::max(1, dense->tiles)) : sms;
     return launch_pdl(grouped_gemm_tc<false>, dim3(grid), dim3(kThreads), kSmemBytes, st, a0, b0,
                       a1, b1, args);
   }
-  return launch_pdl_cluster2(grouped_gemm_tc<true>, dim3(num_sms & ~1), dim3(kThreads),
+  const int pairs = dense ? std::min(sms / 2, std::max(1, dense->tiles)) : sms / 2;
+  return launch_pdl_cluster2(grouped_gemm_tc<true>, dim3(2 * std::max(1, pairs)), dim3(kThreads),
                              kSmemBytes, st, a0, b0, a1, b1, args);
 }
 

@@ -46,11 +46,13 @@ struct DenseTiling {
 };
 
 // pair: tiles of 256 weight rows on two-CTA clusters (tile list built with
-// 256-row weight blocks); otherwise 128 weight rows per CTA.
+// 256-row weight blocks, or dense m_tiles of 256 rows); otherwise 128 weight
+// rows per CTA. max_ctas > 0 caps the persistent grid (the rest of the SMs
+// stay free for work on another stream).
 cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& shared, int E,
                                    bool gelu, const Tile* tiles, const int* n_tiles,
                                    const DenseTiling* dense, bool pair, uint32_t* status,
-                                   int num_sms, cudaStream_t st);
+                                   int num_sms, cudaStream_t st, int max_ctas = 0);
 
 cudaError_t launch_gate_logits(const moe_layer_desc& d, const void* x, const void* wr,
                                float* logits, cudaStream_t st);
@@ -63,9 +65,12 @@ cudaError_t launch_topk_select(const moe_layer_desc& d, const float* logits, int
 cudaError_t launch_gate_logits_tc(const moe_layer_desc& d, const WsLayout& L, char* ws,
                                   const void* x, const void* wr, float* parts, int num_sms,
                                   cudaStream_t st);
+// shared_tiles = false: the tile lists leave the shared expert out (it runs
+// in launches of its own).
 cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws,
                             const int32_t* idx, int32_t* counts, int32_t* offsets,
-                            int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st);
+                            int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st,
+                            bool shared_tiles = true);
 cudaError_t launch_dispatch_scratch(const moe_layer_desc& d, int n_chunks, int32_t* hist,
                                    int32_t* base, WsHeader* hdr, const int32_t* idx,
                                    int32_t* counts, int32_t* offsets, int32_t* perm,
