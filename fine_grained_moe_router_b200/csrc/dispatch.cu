@@ -42,7 +42,8 @@ __global__ void __launch_bounds__(256) chunk_histogram(const int32_t* __restrict
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)blockIdx.x * E + e] = h[e];
 }
 
-// Block-wide exclusive scan of one int per thread (blockDim.x == 1024).
+// Block-wide exclusive scan of one int per thread (blockDim.x a multiple of
+// 32, at most 1024).
 __device__ int block_exclusive_scan(int v, int* sh, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
@@ -331,22 +332,24 @@ __global__ void __launch_bounds__(256) chunk_scatter(const int32_t* __restrict__
 // scatter of the three kernels above, without their two launch gaps. Warp w
 // owns the consecutive copies [w * per_warp, (w + 1) * per_warp); counts per
 // (warp, expert) live in dynamic shared memory (32 * E ints, twice).
-constexpr int kSmallWarps = 32;
+constexpr int kSmallWarps = 32;   // warps of the one-CTA dispatch (at most)
 
-// The whole dispatch of at most kChunk copies by one CTA of 1024 threads
-// (dyn_smem: 2 * kSmallWarps * E ints).
+// The whole dispatch of at most kChunk copies by one CTA of more than E
+// threads (a multiple of 32; dyn_smem: 2 * (blockDim / 32) * E ints). Each
+// warp counts and places a contiguous range of the copies.
 __device__ void dispatch_block(const int32_t* __restrict__ idx, int TK, int E, int T,
                                int has_shared, int32_t* __restrict__ counts,
                                int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
                                int32_t* __restrict__ inv, const TileSpec& ts,
                                WsHeader* __restrict__ hdr, int* dyn_smem) {
-  int* cnt = dyn_smem;                      // [kSmallWarps][E]
-  int* pre = dyn_smem + kSmallWarps * E;    // [kSmallWarps][E]
+  const int nw = blockDim.x >> 5;
+  int* cnt = dyn_smem;             // [nw][E]
+  int* pre = dyn_smem + nw * E;    // [nw][E]
   __shared__ int sh[96];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) cnt[i] = 0;
+  for (int i = threadIdx.x; i < nw * E; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
-  const int per_warp = (TK + kSmallWarps - 1) / kSmallWarps;
+  const int per_warp = (TK + nw - 1) / nw;
   const int w0 = min(TK, warp * per_warp), w1 = min(TK, w0 + per_warp);
   bool bad = false;
   for (int i = w0 + lane; i < w1; i += 32) {
@@ -358,17 +361,17 @@ __device__ void dispatch_block(const int32_t* __restrict__ idx, int TK, int E, i
   }
   if (bad) atomicOr(&hdr->status, kStatusBadIndex);
   __syncthreads();
-  const int e = threadIdx.x;   // one thread per expert slot (E <= 512 < 1024)
+  const int e = threadIdx.x;   // one thread per expert slot (blockDim > E)
   int c = 0;
   if (e < E)
-    for (int w = 0; w < kSmallWarps; ++w) c += cnt[w * E + e];
+    for (int w = 0; w < nw; ++w) c += cnt[w * E + e];
   int total;
   const int off = block_exclusive_scan(e < E ? c : 0, sh, &total);
   if (e < E) {
     counts[e] = c;
     offsets[e] = off;
     int run = off;
-    for (int w = 0; w < kSmallWarps; ++w) {
+    for (int w = 0; w < nw; ++w) {
       pre[w * E + e] = run;
       run += cnt[w * E + e];
       cnt[w * E + e] = 0;
@@ -409,25 +412,27 @@ __global__ void __launch_bounds__(1024) dispatch_small(const int32_t* __restrict
 }
 
 // Gather of dispatched activation rows: xp[row] = x[perm[row] / K] (bf16,
-// 16-byte vectors), so the tensor-core GEMM reads contiguous rows.
+// 16-byte vectors), so the tensor-core GEMM reads contiguous rows. One warp
+// per row; each lane issues up to 16 vector loads before its first store
+// (a 4096-wide row in one memory round trip).
 __global__ void __launch_bounds__(256) gather_rows(const uint4* __restrict__ x,
                                                    const int32_t* __restrict__ perm, int TK,
                                                    int K, int row_vecs, uint4* __restrict__ xp) {
   pdl_wait();
   pdl_trigger();
-  // one warp per row, 16-byte vectors, four in flight per lane
+  constexpr int kVecs = 16;   // vectors in flight per lane
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < TK; row += warps) {
     const uint4* src = x + (size_t)(perm[row] / K) * row_vecs;
     uint4* dst = xp + (size_t)row * row_vecs;
-    for (int v0 = lane; v0 < row_vecs; v0 += 128) {
-      uint4 a[4];
+    for (int v0 = lane; v0 < row_vecs; v0 += 32 * kVecs) {
+      uint4 a[kVecs];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < kVecs; ++q)
         if (v0 + 32 * q < row_vecs) a[q] = src[v0 + 32 * q];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < kVecs; ++q)
         if (v0 + 32 * q < row_vecs) dst[v0 + 32 * q] = a[q];
     }
   }
@@ -463,6 +468,9 @@ cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws
   const TileSpec ts = make_tile_spec(d, L, ws, tc_tiles, /*split=*/true);
   const int has_shared = (d.Ds > 0 && shared_tiles) ? 1 : 0;
   if (TK > 0 && TK <= kChunk) {
+    // all 32 warps even for a handful of copies: they share the writing of
+    // the tile lists (thousands of tiles for a few experts with a wide D)
+    const int threads = 32 * kSmallWarps;
     const size_t smem = sizeof(int) * 2 * kSmallWarps * (size_t)d.E;
     static bool attr_set[64] = {false};   // per device: dynamic smem above 48 KB
     int dev = 0;
@@ -474,7 +482,7 @@ cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws
       if (e != cudaSuccess) return e;
       if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    return launch_pdl(dispatch_small, dim3(1), dim3(1024), smem, st, idx, TK, d.E, d.T,
+    return launch_pdl(dispatch_small, dim3(1), dim3(threads), smem, st, idx, TK, d.E, d.T,
                       has_shared, counts, offsets, perm, inv, ts, hdr);
   }
   cudaError_t e = cudaSuccess;

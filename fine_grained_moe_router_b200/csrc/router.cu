@@ -108,8 +108,9 @@ __device__ __forceinline__ void select_row(const float* __restrict__ lrow, int n
   const int lane = threadIdx.x & 31;
   // Sum of the n_parts partial logits (reduction splits of the gate GEMM)
   // in split order. The loads of kPB parts for all NJ slots are issued
-  // before any add, so the partial sums cost one round trip per kPB parts.
-  constexpr int kPB = (NJ >= 8) ? 4 : (NJ >= 4 ? 8 : 16);
+  // before any add, so the partial sums cost one round trip per kPB parts
+  // (the router uses at most 16 splits).
+  constexpr int kPB = (NJ >= 16) ? 4 : (NJ >= 8 ? 8 : 16);
   float l[NJ];
 #pragma unroll
   for (int j = 0; j < NJ; ++j) {
