@@ -91,35 +91,20 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   const int t = blockIdx.x;
   const int h = (blockIdx.y * blockDim.x + threadIdx.x) * V::N;
   if (t >= T_ || h >= H) return;
-  // the token's K rows and weights first, then the rows' values four copies
-  // at a time, so a decode step pays a few memory round trips, not K
-  int row[kMaxK];
-  float wk[kMaxK];
-#pragma unroll
-  for (int k = 0; k < kMaxK; ++k)
-    if (k < K) {
-      row[k] = inv[(size_t)t * K + k];
-      wk[k] = w[(size_t)t * K + k];
-    }
   float acc[V::N];
 #pragma unroll
   for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
+  for (int k = 0; k < K; ++k) {
+    const int row = inv[(size_t)t * K + k];
+    const float wk = w[(size_t)t * K + k];
+    const float* src = y_rows + (size_t)row * H + h;
 #pragma unroll
-  for (int k0 = 0; k0 < kMaxK; k0 += 4) {
-    if (k0 >= K) break;
-    float v[4][V::N];
+    for (int q = 0; q < V::N; q += F::N) {
+      float v[F::N];
+      load_parts<F::N>(src + q, rows_parts, rows_stride, v);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (k0 + q < K) {
-        const float* src = y_rows + (size_t)row[k0 + q] * H + h;
-#pragma unroll
-        for (int c = 0; c < V::N; c += F::N) load_parts<F::N>(src + c, rows_parts, rows_stride, v[q] + c);
-      }
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (k0 + q < K)
-#pragma unroll
-        for (int i = 0; i < V::N; ++i) acc[i] = fmaf(wk[k0 + q], v[q][i], acc[i]);
+      for (int i = 0; i < F::N; ++i) acc[q + i] = fmaf(wk, v[i], acc[q + i]);
+    }
   }
   if (y_shared) {
     const float* src = y_shared + (size_t)t * H + h;
