@@ -82,6 +82,7 @@ struct TileSpec {
   int splits1_routed, splits1_shared;     // reduction splits of GEMM1 tiles
   int splits2_routed, splits2_shared;     // reduction splits of GEMM2 tiles
   int mtile;                              // weight rows per tile: 128, or 256 on CTA pairs
+  int lpt;                                // 1: experts by descending rows; 0: by index
 };
 
 // Number of balanced row tiles for a group of c rows and the rows per tile
@@ -125,7 +126,10 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
   // times weight-row blocks (128, or 256 on CTA pairs) times reduction
   // splits. Order: the shared expert first, then the routed experts by
   // descending row count (ties by index), so the longest work starts first;
-  // the order inside a group is given where the tiles are written.
+  // the order inside a group is given where the tiles are written. Batches
+  // of at most 4 copies per expert on average keep the experts in index
+  // order instead: their tiles all cost about one weight slab, and the
+  // O(E) ranking is a visible part of a decode step.
   __shared__ int s_cnt[kMaxE];
   __shared__ int s_pos1[kMaxE], s_pos2[kMaxE];
   __shared__ int s_first1[kMaxE + 1], s_first2[kMaxE + 1], s_nt[kMaxE + 1], s_rper[kMaxE + 1],
@@ -141,9 +145,13 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
   __syncthreads();
   int rank = 0;
   if (e < E) {
-    for (int q = 0; q < E; ++q) {
-      const int cq = s_cnt[q];
-      rank += (cq > c) || (cq == c && q < e);
+    if (ts.lpt) {
+      for (int q = 0; q < E; ++q) {
+        const int cq = s_cnt[q];
+        rank += (cq > c) || (cq == c && q < e);
+      }
+    } else {
+      rank = e;
     }
     s_pos1[rank] = nt_rows * mt1 * ts.splits1_routed;   // tile counts in rank order
     s_pos2[rank] = nt_rows * ts.m_tiles2 * ts.splits2_routed;
@@ -446,6 +454,7 @@ static TileSpec make_tile_spec(const moe_layer_desc& d, const WsLayout& L, char*
   ts.tc1 = tc_tiles ? reinterpret_cast<Tile*>(ws + L.tiles_tc1) : nullptr;
   ts.tc2 = tc_tiles ? reinterpret_cast<Tile*>(ws + L.tiles_tc2) : nullptr;
   ts.mtile = (split && L.sp.pair) ? 256 : 128;
+  ts.lpt = ((long long)d.T * d.K > 4LL * d.E) ? 1 : 0;
   ts.m_tiles1_routed = d.D / ts.mtile;
   ts.m_tiles1_shared = d.Ds / ts.mtile;
   ts.m_tiles2 = d.H / ts.mtile;
