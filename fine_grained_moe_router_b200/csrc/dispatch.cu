@@ -109,8 +109,8 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
   const int g_rows = (e < E) ? c : ((e == E && has_shared) ? T : 0);
   const int r_base = (e < E) ? off : 0;
   const int nt_simt = (g_rows + kSimtRows - 1) / kSimtRows;
-  int tot_simt;
-  const int first_simt = block_exclusive_scan(nt_simt, sh, &tot_simt);
+  int tot_simt = 0, first_simt = 0;
+  if (ts.simt) first_simt = block_exclusive_scan(nt_simt, sh, &tot_simt);   // uniform branch
   if (ts.simt) {
     for (int i = 0; i < nt_simt; ++i) {
       Tile t;
