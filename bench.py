@@ -109,27 +109,85 @@ def roofline_bound(flops, nbytes, peaks):
 
 # --------------------------------------------------------------- clocks ---
 class ClockSampler:
+    """SM clock and clock-event reasons of the benchmarked GPU during the timed
+    region. Polls NVML from a thread every few milliseconds (a timed region
+    of a few tens of milliseconds still gets samples); falls back to
+    `nvidia-smi -lms 200` when NVML is not importable. Reads only."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device: torch.device):
+        self.device = device
         self.proc = None
         self.path = None
+        self.thread = None
+        self.samples = []
+        self.max_mhz = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            try:
+                u = str(uuid)
+                return pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+            except Exception:
+                pass
+        bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+        return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def start(self):
+        import threading
+        try:
+            import pynvml
+            h = self._nvml_handle()
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.stop_flag = threading.Event()
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((float(mhz), int(rs)))
+                    except Exception:
+                        pass
+                    time.sleep(0.002)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            while not self.samples and self.thread.is_alive():   # first sample before timing
+                time.sleep(0.001)
+            return
+        except Exception:
+            self.thread = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
+            idx = self.device.index if self.device.index is not None else 0
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.gpu), "-f", self.path],
+                 "-lms", "200", "-i", str(idx), "-f", self.path],
                 stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"],
+                        "source": "nvml"}
+            reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS if r & bit})
+            return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                    "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                    "samples": len(self.samples), "source": "nvml"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.25)
@@ -151,7 +209,7 @@ class ClockSampler:
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": "nvidia-smi"}
 
 
 def build_and_import():
@@ -289,12 +347,14 @@ class Runner:
     def step(self):
         self.M.moe_layer_forward(self.desc, self.weights, self.x, self.y, self.routing, self.ws)
 
-    def timed(self, steps, warmup, world, device, stage_events=False):
+    def timed(self, steps, warmup, world, device, sampler=None):
         for _ in range(warmup):
             self.step()
         torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
+        if sampler is not None:
+            sampler.start()   # clocks of the timed region only
         n0 = self.M.moe_kernel_launch_count()
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         start.record()
@@ -303,6 +363,8 @@ class Runner:
         end.record()
         torch.cuda.synchronize()
         launches = self.M.moe_kernel_launch_count() - n0
+        if sampler is not None:
+            self.clocks = sampler.stop()
         barrier(world)
         ms = max_over_ranks(start.elapsed_time(end), world, device)
         return ms, launches
@@ -387,10 +449,8 @@ def run_ours(args, wl, T):
     dev = {k: (v.to(device) if v is not None else None) for k, v in host.items()}
     R = Runner(M, wl, dev, T, replica=rank)
 
-    sampler = ClockSampler(device.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
-    sampler.start()
-    ms, launches = R.timed(args.steps, args.warmup, world, device)
-    clocks = sampler.stop()
+    ms, launches = R.timed(args.steps, args.warmup, world, device, sampler=ClockSampler(device))
+    clocks = R.clocks
     ms_step = ms / args.steps
     value = world * T * args.steps / (ms / 1e3)
 
