@@ -107,21 +107,22 @@ static Splits compute_splits(const moe_layer_desc& d) {
   const long long row_tiles = (T + kTcRows - 1) / kTcRows;
   s.router = std::min(16, split_count(row_tiles * ((d.E + 127) / 128), d.H / 64, 148, 2));
   s.router = normalise_splits(d.H / 64, s.router);   // no empty split after the cap
-  // Each touched expert has at least one row tile; a decode step touches
-  // min(E, T*K) experts.
+  // Routed row tiles: each touched expert has at least one. A batch touches
+  // between K and min(E, T*K) experts (all of them once it holds several
+  // copies per expert); the model averages over that range.
   const long long r_rows = std::max(touched, (TK + kTcRows - 1) / kTcRows);
+  const long long r_lo = (TK >= 8LL * d.E) ? r_rows
+                         : std::max<long long>(d.K + (touched - d.K) / 2,
+                                               (TK + kTcRows - 1) / kTcRows);
   if (!s.pair) {
     // Weight-streaming regime: balance both expert GEMMs over the SMs. The
     // first GEMM's splits are added up by the last split of each tile, one
-    // round of loads per few rows, so they are used for short tiles only:
-    // at most kFixupRows rows per routed expert on average, or per shared tile.
+    // round of loads per few rows, so they are used for short tiles only
+    // (at most kFixupRows rows per routed expert on average, or per shared
+    // tile) and their fixed cost per tile is higher.
     constexpr int kFixupRows = 16;
     const int max_r1 = (TK <= kFixupRows * touched) ? 16 : 1;
     const int max_s1 = (T <= kFixupRows) ? 16 : 1;
-    // Fixed cost per tile, in reduction blocks: the first layer's splits
-    // also pay the partial round trip and the fixup.
-    // a batch touches between K and min(E, T*K) experts
-    const long long r_lo = std::max<long long>(d.K + (touched - d.K) / 2, (TK + kTcRows - 1) / kTcRows);
     pick_splits(r_lo * (d.D / 128), r_rows * (d.D / 128), d.H / 64,
                 d.Ds ? row_tiles * (d.Ds / 128) : 0, d.H / 64, 148, max_r1, max_s1, 6.0,
                 &s.gemm1_routed, &s.gemm1_shared);
@@ -130,18 +131,12 @@ static Splits compute_splits(const moe_layer_desc& d) {
                 &s.gemm2_routed, &s.gemm2_shared);
     return s;
   }
-  // CTA pairs: split the second GEMM only when it has fewer tiles than pairs
-  constexpr int kTargetTiles = 148;
+  // CTA pairs: the second GEMM's splits from the same model over the 74
+  // pairs (its partials are added by the combine); the first layer stays
+  // unsplit on pairs.
   const int mt2 = d.H / 256;
-  const long long r_tiles = r_rows * mt2;
-  const long long s_tiles = d.Ds ? row_tiles * mt2 : 0;
-  if (r_tiles + s_tiles < kTargetTiles) {
-    const int kbr = d.D / 64, kbs = d.Ds / 64;
-    const long long total_kb = r_tiles * kbr + s_tiles * kbs;
-    const int per = (int)std::max<long long>(4, (total_kb + kTargetTiles - 1) / kTargetTiles);
-    s.gemm2_routed = split_count(1, kbr, (kbr + per - 1) / per, 4);
-    if (d.Ds) s.gemm2_shared = split_count(1, kbs, (kbs + per - 1) / per, 4);
-  }
+  pick_splits(r_lo * mt2, r_rows * mt2, d.D / 64, d.Ds ? row_tiles * mt2 : 0,
+              d.Ds ? d.Ds / 64 : 0, 74, 16, 16, 2.0, &s.gemm2_routed, &s.gemm2_shared);
   return s;
 }
 
