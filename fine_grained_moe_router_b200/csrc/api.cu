@@ -243,15 +243,17 @@ static moe_status check_ptrs(std::initializer_list<const void*> ps) {
 }
 
 static int num_sms() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (!n) {
     int v = 0;
     cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = v > 0 ? v : 148;
+    n = v > 0 ? v : 148;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 #define MOE_TRY(expr)                 \

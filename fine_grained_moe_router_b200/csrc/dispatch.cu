@@ -13,6 +13,8 @@
 //   3. chunk_scatter     stable placement: inside a chunk, warps own
 //                        consecutive copy ranges and rank equal experts with
 //                        __match_any_sync, so the order is ascending copy id.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "launch.cuh"
@@ -481,15 +483,15 @@ cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws
     // the tile lists (thousands of tiles for a few experts with a wide D)
     const int threads = 32 * kSmallWarps;
     const size_t smem = sizeof(int) * 2 * kSmallWarps * (size_t)d.E;
-    static bool attr_set[64] = {false};   // per device: dynamic smem above 48 KB
+    static std::atomic<bool> attr_set[64];   // per device: dynamic smem above 48 KB
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
       e = cudaFuncSetAttribute(dispatch_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(sizeof(int) * 2 * kSmallWarps * kMaxE));
       if (e != cudaSuccess) return e;
-      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+      if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
     }
     return launch_pdl(dispatch_small, dim3(1), dim3(threads), smem, st, idx, TK, d.E, d.T,
                       has_shared, counts, offsets, perm, inv, ts, hdr);
