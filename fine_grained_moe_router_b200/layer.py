@@ -59,13 +59,18 @@ class MoELayer:
         }
 
     def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, routing: Optional[dict] = None,
-                stream=None) -> torch.Tensor:
-        """y = MoE(x) for x [T, H]; fills `routing` (see routing_buffers) if given."""
+                stream=None, gumbel_noise: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """y = MoE(x) for x [T, H]; fills `routing` (see routing_buffers) if given.
+        gumbel_noise [T, E] fp32: noisy routing (Gumbel draws added to l + B)."""
         T = x.shape[0]
         if y is None:
             y = torch.empty_like(x)
         r = B.make_routing(**routing) if routing is not None else None
-        B.moe_layer_forward(self.desc(T), self.weights, x, y, r, self.workspace(T), stream)
+        if gumbel_noise is None:
+            B.moe_layer_forward(self.desc(T), self.weights, x, y, r, self.workspace(T), stream)
+        else:
+            B.moe_layer_forward_noisy(self.desc(T), self.weights, x, gumbel_noise, y, r,
+                                      self.workspace(T), stream)
         return y
 
     __call__ = forward
@@ -73,3 +78,10 @@ class MoELayer:
     def stats(self, counts: torch.Tensor, T: int, straggler_mask: Optional[torch.Tensor] = None,
               stream=None) -> dict:
         return B.moe_expert_stats(self.desc(T), counts, straggler_mask, self.workspace(T), stream)
+
+    def update_bias(self, counts: torch.Tensor, tokens: int, gamma: float, stream=None) -> None:
+        """Dynamic bias update from expert counts accumulated over `tokens`
+        tokens: B_e -= gamma for overloaded experts, += gamma for idle ones."""
+        if self.tensors[5] is None:
+            raise ValueError("the layer has no expert bias tensor to update")
+        B.moe_bias_update(self.desc(tokens), counts, self.tensors[5], gamma, stream)
