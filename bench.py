@@ -402,30 +402,58 @@ class Runner:
         return out
 
     def e2e(self, steps, warmup, world, device):
-        """Through the public API from pinned host memory: H2D of x, forward,
-        D2H of y, every step."""
+        """Through the public API from pinned host memory: every step copies its
+        x host -> device, runs the forward and copies its y device -> host, all
+        inside the timed region. As a serving loop would, the copies run on a
+        second stream with double-buffered device tensors, so step i+1's input
+        copy and step i-1's output copy overlap step i's forward."""
         xh = self.x_host.pin_memory()
-        yh = torch.empty_like(xh).pin_memory()
+        yh = [torch.empty_like(xh).pin_memory() for _ in range(2)]
+        xd = [self.x, torch.empty_like(self.x)]
+        yd = [self.y, torch.empty_like(self.y)]
+        comp = torch.cuda.current_stream()
+        copy = torch.cuda.Stream()
+        ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("h2d", "fwd", "d2h")}
+        M = self.M
 
-        def one():
-            self.x.copy_(xh, non_blocking=True)
-            self.step()
-            yh.copy_(self.y, non_blocking=True)
+        def run(n, start=None):
+            if start is not None:
+                start.record(comp)
+            copy.wait_stream(comp)
+            with torch.cuda.stream(copy):
+                xd[0].copy_(xh, non_blocking=True)
+                ev["h2d"][0].record(copy)
+            for i in range(n):
+                b = i % 2
+                comp.wait_event(ev["h2d"][b])
+                if i >= 2:
+                    comp.wait_event(ev["d2h"][b])        # y buffer b has left for the host
+                M.moe_layer_forward(self.desc, self.weights, xd[b], yd[b], self.routing, self.ws,
+                                    comp)
+                ev["fwd"][b].record(comp)
+                with torch.cuda.stream(copy):
+                    if i + 1 < n:
+                        nb = (i + 1) % 2
+                        if i >= 1:
+                            copy.wait_event(ev["fwd"][nb])   # x buffer nb is no longer read
+                        xd[nb].copy_(xh, non_blocking=True)
+                        ev["h2d"][nb].record(copy)
+                    copy.wait_event(ev["fwd"][b])
+                    yh[b].copy_(yd[b], non_blocking=True)
+                    ev["d2h"][b].record(copy)
+            comp.wait_stream(copy)
 
-        for _ in range(warmup):
-            one()
+        run(warmup)
         torch.cuda.synchronize()
         barrier(world)
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        start.record()
-        for _ in range(steps):
-            one()
-        end.record()
+        run(steps, start)
+        end.record(comp)
         torch.cuda.synchronize()
         barrier(world)
         ms = max_over_ranks(start.elapsed_time(end), world, device)
         nbytes = xh.numel() * xh.element_size()
-        return ms, nbytes, yh.numel() * yh.element_size()
+        return ms, nbytes, yh[0].numel() * yh[0].element_size()
 
     def touched(self):
         return int((self.counts > 0).sum().item())
