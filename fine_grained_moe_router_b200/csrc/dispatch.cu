@@ -102,6 +102,8 @@ __device__ __forceinline__ void tc_row_split(int c, int* nt, int* rows) {
   *rows = r;
 }
 
+constexpr int kFlatTileList = 8192;   // tiles above which every thread shares the writing
+
 // Writes the tile lists of every group; thread e < E owns expert e (c rows
 // starting at row `off`), thread E owns the shared expert (T token rows).
 __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const TileSpec& ts,
@@ -133,7 +135,7 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
   // order instead: their tiles all cost about one weight slab, and the
   // O(E) ranking is a visible part of a decode step.
   __shared__ int s_cnt[kMaxE];
-  __shared__ int s_pos1[kMaxE], s_pos2[kMaxE];
+  __shared__ int s_pos1[kMaxE], s_pos2[kMaxE], s_grp[kMaxE];
   __shared__ int s_first1[kMaxE + 1], s_first2[kMaxE + 1], s_nt[kMaxE + 1], s_rper[kMaxE + 1],
       s_rows[kMaxE + 1], s_rbase[kMaxE + 1];
   int nt_rows, rows_per;
@@ -155,6 +157,7 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
     } else {
       rank = e;
     }
+    s_grp[rank] = e;
     s_pos1[rank] = nt_rows * mt1 * ts.splits1_routed;   // tile counts in rank order
     s_pos2[rank] = nt_rows * ts.m_tiles2 * ts.splits2_routed;
   }
@@ -177,26 +180,62 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
   }
   __syncthreads();
   if (ts.tc1) {
+    const int n1_all = sh1 + tot1, n2_all = sh2 + tot2;
+    // Long lists (a long batch: thousands of tiles in the shared expert's or
+    // a hot expert's group) are spread over all threads, each finding its
+    // tile's group by binary search over the groups' first positions;
+    // shorter ones go one group per warp, which needs no search.
+    const bool flat = n1_all + n2_all > kFlatTileList;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-    for (int g = warp; g <= E; g += nwarps) {
-      const int nt = s_nt[g];
-      if (nt == 0) continue;
-      const int m1 = (g < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared;
-      const int sp1 = (g < E) ? ts.splits1_routed : ts.splits1_shared;
-      const int sp2 = (g < E) ? ts.splits2_routed : ts.splits2_shared;
-      const int n1 = nt * m1 * sp1, n2 = nt * ts.m_tiles2 * sp2;
-      for (int i = lane; i < n1 + n2; i += 32) {
-        const bool first = i < n1;
-        const int j = first ? i : i - n1;
-        const int sp = first ? sp1 : sp2;
-        const int mt = first ? m1 : ts.m_tiles2;
+    int g = flat ? 0 : warp, i_begin = flat ? threadIdx.x : lane;
+    const int i_step = flat ? (int)blockDim.x : 32;
+    while (g <= E) {
+      // tiles of group g (per-warp mode) or of both whole lists (flat mode)
+      const int nt_g = s_nt[g];
+      const int m1_g = (g < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared;
+      const int sp1_g = (g < E) ? ts.splits1_routed : ts.splits1_shared;
+      const int sp2_g = (g < E) ? ts.splits2_routed : ts.splits2_shared;
+      const int n_items = flat ? n1_all + n2_all : nt_g * (m1_g * sp1_g + ts.m_tiles2 * sp2_g);
+      for (int i = i_begin; i < n_items; i += i_step) {
+        int gg = g, j;
+        bool first;
+        if (flat) {
+          first = i < n1_all;
+          const int li = first ? i : i - n1_all;   // position in its list
+          const int shn = first ? sh1 : sh2;
+          if (li < shn) {
+            gg = E;
+            j = li;
+          } else {
+            const int k = li - shn;
+            const int* pos = first ? s_pos1 : s_pos2;
+            int lo = 0, hi = E - 1;   // last rank position with pos <= k (a non-empty group)
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (pos[mid] <= k)
+                lo = mid;
+              else
+                hi = mid - 1;
+            }
+            gg = s_grp[lo];
+            j = k - pos[lo];
+          }
+        } else {
+          const int n1 = nt_g * m1_g * sp1_g;
+          first = i < n1;
+          j = first ? i : i - n1;
+        }
+        const int nt = s_nt[gg];
+        const int sp = first ? ((gg < E) ? ts.splits1_routed : ts.splits1_shared)
+                             : ((gg < E) ? ts.splits2_routed : ts.splits2_shared);
+        const int mt = first ? ((gg < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared) : ts.m_tiles2;
         // Order inside the group: when the group has more activation rows than
         // weight rows the row blocks are outermost (the weight matrix stays in
         // L2 while the rows stream once); otherwise the weight blocks are
         // outermost (each weight slab streams once while its row blocks, on
         // neighbouring CTAs, reuse it from L2). Splits vary fastest after that.
-        int r, q, j0;   // j0: the list position of the split-0 tile of j
-        const bool row_outer = s_rows[g] > mt * ts.mtile;
+        int r, q, j0;   // j0: the position of the split-0 tile of j in the group
+        const bool row_outer = s_rows[gg] > mt * ts.mtile;
         if (row_outer) {
           r = j / (mt * sp);
           q = j - r * (mt * sp);
@@ -205,22 +244,24 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
           q = j / nt;
         }
         Tile t;
-        t.g = g;
-        t.r0 = s_rbase[g] + r * s_rper[g];
-        t.n = min(s_rper[g], s_rows[g] - r * s_rper[g]);
+        t.g = gg;
+        t.r0 = s_rbase[gg] + r * s_rper[gg];
+        t.n = min(s_rper[gg], s_rows[gg] - r * s_rper[gg]);
         t.m0 = (q / sp) * ts.mtile;
         t.ks = q % sp;
         j0 = row_outer ? j - t.ks : j - t.ks * nt;
         t.arrivals[0] = 0;
         t.arrivals[1] = 0;
         if (first) {
-          t.first_split = s_first1[g] + j0;
-          ts.tc1[s_first1[g] + j] = t;
+          t.first_split = s_first1[gg] + j0;
+          ts.tc1[s_first1[gg] + j] = t;
         } else {
-          t.first_split = s_first2[g] + j0;
-          ts.tc2[s_first2[g] + j] = t;
+          t.first_split = s_first2[gg] + j0;
+          ts.tc2[s_first2[gg] + j] = t;
         }
       }
+      if (flat) break;
+      g += nwarps;
     }
   }
   if (threadIdx.x == 0) {
