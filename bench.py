@@ -84,19 +84,52 @@ def algorithmic(wl, T, touched, counts=None):
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the two
 # expert-GEMM launches of one step, from one ncu capture of this workload
-# (profiles/grouped_gemm_tc_mixtral_T4096.md). Valid only for the kernel
-# source it was measured on: any change to that file makes it null.
-MEASURED_TRAFFIC = {"kernel_sha256_16": "e993bb6d127b2a7a", "workload": "c2", "T": 4096,
+# (profiles/grouped_gemm_tc_mixtral_T4096.md). Valid only for the kernel code
+# it was measured on: the key is a fingerprint of the GEMM source and the
+# headers it includes with comments and whitespace removed, so any change to
+# the code (not to its comments) makes it null.
+MEASURED_TRAFFIC = {"kernel_code_sha256_16": "d36ae6b1c4a34f7c", "workload": "c2", "T": 4096,
                     "bytes_per_step": 1.103e9 + 0.236e9 + 1.646e9 + 0.135e9}
+TRAFFIC_SOURCES = ("ffn_tc.cu", "common.cuh", "kernels.cuh")
+
+
+def _strip_c_comments(text):
+    """C/C++ source without comments or whitespace (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            if not c.isspace():
+                out.append(c)
+            i += 1
+    return "".join(out)
+
+
+def kernel_code_fingerprint():
+    import hashlib
+    h = hashlib.sha256()
+    for name in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "fine_grained_moe_router_b200", "csrc", name)) as f:
+            h.update(_strip_c_comments(f.read()).encode())
+    return h.hexdigest()[:16]
 
 
 def measured_traffic(wl, T):
-    import hashlib
-    src = os.path.join(ROOT, "fine_grained_moe_router_b200", "csrc", "ffn_tc.cu")
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()[:16]
     m = MEASURED_TRAFFIC
-    if sha == m["kernel_sha256_16"] and wl.key == m["workload"] and T == m["T"]:
+    if (kernel_code_fingerprint() == m["kernel_code_sha256_16"] and wl.key == m["workload"]
+            and T == m["T"]):
         return m["bytes_per_step"] / 2.0   # mean per launch of the two expert GEMMs
     return None
 

@@ -13,6 +13,9 @@
 //   3. chunk_scatter     stable placement: inside a chunk, warps own
 //                        consecutive copy ranges and rank equal experts with
 //                        __match_any_sync, so the order is ascending copy id.
+// Batches of at most one chunk (kChunk copies) run all three steps in one CTA
+// (dispatch_small). gather_rows then copies the dispatched activation rows
+// for the tensor-core GEMMs.
 #include <atomic>
 
 #include "common.cuh"

@@ -3,10 +3,12 @@
 // One launch computes every tile of one of the two expert layers ("MoE
 // architecture in production" §3.1: Linear -> GeLU -> Linear per expert),
 // for all routed experts plus the shared expert, from a device-side tile list
-// written by the dispatch step. A tile is 128 weight rows (the MMA M side) by
-// up to 256 dispatched activation rows (the MMA N side, rounded up to 16):
-// weights are the A operand and tokens the B operand, so a decode step with a
-// handful of rows per expert still fills the 128-row MMA and the kernel
+// written by the dispatch step (or a dense tiling: the gate GEMM, and the
+// shared expert when it runs on its own stream). A tile is 128 weight rows
+// (the MMA M side; 256 on a CTA pair) by up to 256 dispatched activation
+// rows (the MMA N side, rounded up to 16), optionally one reduction split of
+// them: weights are the A operand and tokens the B operand, so a decode step
+// with a handful of rows per expert still fills the MMA and the kernel
 // streams each touched weight slab once.
 //
 // Per CTA (persistent, one per SM, 320 threads):
@@ -18,7 +20,9 @@
 //           epilogue of one tile overlaps the MMAs of the next
 //   warps 0-7  epilogue: tcgen05.ld of the accumulator (thread = weight row,
 //           two warps per TMEM lane quarter splitting the columns), exact
-//           GeLU for the first layer, stores into row-major output
+//           GeLU for the first layer, stores into row-major output; a split
+//           first-layer tile stores fp32 partials and its last split adds
+//           them up before the GeLU
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // kStatusTimeout in the workspace, drains its in-flight copies and MMAs,
 // frees its TMEM and returns.
