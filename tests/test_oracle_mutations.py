@@ -16,7 +16,8 @@ import test_oracle_pins as pins
 
 _orig = {n: getattr(om, n) for n in ("select_topk", "dispatch", "gelu_erf", "gini_exact",
                                       "capacity", "load_stats", "expert_ffn", "selection_scores",
-                                      "moe_layer_forward")}
+                                      "moe_layer_forward", "bias_update", "expert_offsets",
+                                      "combine")}
 
 
 def _topk_high_index_ties(logits, bias, K, noise=None):
@@ -112,6 +113,43 @@ def _stats_overflow_counts_experts(counts, T, K, cf_num=5, cf_den=4):
     return st
 
 
+def _bias_sign_flipped(bias, counts, T, K, gamma, cf_num=5, cf_den=4):
+    return _orig["bias_update"](bias, counts, T, K, -gamma, cf_num, cf_den)
+
+
+def _bias_overload_at_capacity(bias, counts, T, K, gamma, cf_num=5, cf_den=4):
+    b = np.asarray(bias, np.float32).copy()
+    c = np.asarray(counts, np.int64)
+    cap = om.capacity(T, K, c.size, cf_num, cf_den)
+    g = np.float32(gamma)
+    b[c >= cap] -= g
+    b[c == 0] += g
+    return b
+
+
+def _bias_idle_untouched(bias, counts, T, K, gamma, cf_num=5, cf_den=4):
+    b = np.asarray(bias, np.float32).copy()
+    c = np.asarray(counts, np.int64)
+    b[c > om.capacity(T, K, c.size, cf_num, cf_den)] -= np.float32(gamma)
+    return b
+
+
+def _offsets_inclusive(counts):
+    c = np.asarray(counts, np.int64)
+    return np.concatenate([np.cumsum(c), [c.sum()]]).astype(np.int32)
+
+
+def _combine_unweighted(y_rows, w, inv, y_shared=None):
+    return _orig["combine"](y_rows, np.ones_like(np.asarray(w, np.float64)), inv, y_shared)
+
+
+def _stats_skew_without_epsilon(counts, T, K, cf_num=5, cf_den=4):
+    st = _orig["load_stats"](counts, T, K, cf_num, cf_den)
+    mn = int(np.min(counts))
+    st["skew_ratio"] = float(np.max(counts)) / mn if mn else math.inf
+    return st
+
+
 MUTANTS = {
     "ties_to_higher_index": ("select_topk", _topk_high_index_ties),
     "weights_not_renormalised": ("select_topk", _topk_no_renorm),
@@ -128,6 +166,12 @@ MUTANTS = {
     "overflow_counts_experts": ("load_stats", _stats_overflow_counts_experts),
     "gumbel_noise_ignored": ("selection_scores", _scores_ignore_noise),
     "noisy_weights_from_clean_scores": ("select_topk", _topk_weights_from_clean_scores),
+    "bias_update_sign_flipped": ("bias_update", _bias_sign_flipped),
+    "bias_update_overload_at_capacity": ("bias_update", _bias_overload_at_capacity),
+    "bias_update_idle_untouched": ("bias_update", _bias_idle_untouched),
+    "offsets_inclusive": ("expert_offsets", _offsets_inclusive),
+    "combine_unweighted": ("combine", _combine_unweighted),
+    "skew_without_epsilon": ("load_stats", _stats_skew_without_epsilon),
 }
 
 PIN_TESTS = [
@@ -149,6 +193,11 @@ PIN_TESTS = [
     pins.test_capacity_integer_form_equals_page_float_form,
     pins.test_gumbel_max_picks_each_expert_with_its_softmax_probability,
     pins.test_noisy_weights_are_the_softmax_of_the_noisy_scores,
+    pins.test_combine_worked_example,
+    pins.test_stagewise_grouped_ffn_and_combine_equal_layer_definition,
+    pins.test_bias_update_moves_only_overloaded_and_idle_experts,
+    pins.test_bias_update_is_a_fixed_point_for_an_even_load,
+    pins.test_repeated_bias_updates_even_out_a_skewed_router,
 ]
 
 

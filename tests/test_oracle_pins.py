@@ -368,6 +368,18 @@ def test_stagewise_grouped_ffn_and_combine_equal_layer_definition():
                                rtol=1e-12, atol=1e-13)
 
 
+def test_combine_worked_example():
+    """Two tokens, K = 2, H = 2, by hand: y[t] = sum_k w[t,k] * rows[inv[t*K+k]] + shared[t]."""
+    rows = np.array([[1.0, -1.0], [2.0, 0.0], [3.0, 1.0], [4.0, 2.0]])
+    inv = np.array([2, 0, 3, 1])                  # copy c of token c // 2 sits in row inv[c]
+    w = np.array([[0.25, 0.75], [0.5, 0.5]])
+    shared = np.array([[10.0, 20.0], [30.0, 40.0]])
+    y = oracle.combine(rows, w, inv)
+    np.testing.assert_array_equal(y, [[0.25 * 3 + 0.75 * 1, 0.25 * 1 + 0.75 * -1],
+                                      [0.5 * 4 + 0.5 * 2, 0.5 * 2 + 0.5 * 0]])
+    np.testing.assert_array_equal(oracle.combine(rows, w, inv, shared), y + shared)
+
+
 def test_combine_K1_unit_weight_is_inverse_permutation():
     rng = _rng(42)
     TK, H = 19, 5
