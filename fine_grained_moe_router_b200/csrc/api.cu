@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "dispatch.cuh"
 #include "kernels.cuh"
 
 namespace moe {
@@ -600,9 +601,13 @@ static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer
   MOE_CUDA_TRY(mark(0));
   MOE_TRY(run_router(d, L, w, x, W.w_router, W.expert_bias, idx, tw, R.logits, st, noise));
   MOE_CUDA_TRY(mark(1));
-  MOE_CUDA_TRY(launch_dispatch(d, L, w, idx, counts, offsets, perm, inv, tc, st,
-                               /*shared_tiles=*/side == nullptr));
-  if (tc) MOE_CUDA_TRY(launch_gather_rows(d, x, perm, w + L.xp, num_sms(), st));
+  if (tc)
+    MOE_CUDA_TRY(launch_dispatch_gather(d, L, w, idx, counts, offsets, perm, inv, st,
+                                        /*shared_tiles=*/side == nullptr, x, w + L.xp,
+                                        num_sms()));
+  else
+    MOE_CUDA_TRY(launch_dispatch(d, L, w, idx, counts, offsets, perm, inv, false, st,
+                                 /*shared_tiles=*/side == nullptr));
   MOE_CUDA_TRY(mark(2));
   MOE_TRY(run_grouped_ffn(d, L, w, x, perm, W.w1, W.w2, W.ws1, W.ws2, yr, ys, st,
                           /*split=*/true, ev ? ev + 3 : nullptr, /*with_shared=*/side == nullptr));

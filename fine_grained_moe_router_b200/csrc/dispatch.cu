@@ -15,10 +15,12 @@
 //                        __match_any_sync, so the order is ascending copy id.
 // Batches of at most one chunk (kChunk copies) run all three steps in one CTA
 // (dispatch_small). gather_rows then copies the dispatched activation rows
-// for the tensor-core GEMMs.
+// for the tensor-core GEMMs; for the smallest batches (kFusedGatherCopies)
+// dispatch_small copies them itself.
 #include <atomic>
 
 #include "common.cuh"
+#include "dispatch.cuh"
 #include "kernels.cuh"
 #include "launch.cuh"
 
@@ -452,44 +454,84 @@ __device__ void dispatch_block(const int32_t* __restrict__ idx, int TK, int E, i
   }
 }
 
+// One dispatched activation row, xp[row] = x[perm[row] / K] (bf16 as
+// 16-byte vectors), copied by one warp: each lane issues up to 16 vector
+// loads before its first store (a 4096-wide row in one memory round trip).
+// A copy index outside [0, TK) (left by a dispatch that rejected an
+// out-of-range expert, which it reports in the status word) copies nothing.
+__device__ __forceinline__ void gather_row(const uint4* __restrict__ x,
+                                           const int32_t* __restrict__ perm, int TK, int K,
+                                           int row_vecs, uint4* __restrict__ xp, int row,
+                                           int lane) {
+  constexpr int kVecs = 16;   // vectors in flight per lane
+  const int c = perm[row];
+  if ((unsigned)c >= (unsigned)TK) return;
+  const uint4* src = x + (size_t)(c / K) * row_vecs;
+  uint4* dst = xp + (size_t)row * row_vecs;
+  for (int v0 = lane; v0 < row_vecs; v0 += 32 * kVecs) {
+    uint4 a[kVecs];
+#pragma unroll
+    for (int q = 0; q < kVecs; ++q)
+      if (v0 + 32 * q < row_vecs) a[q] = src[v0 + 32 * q];
+#pragma unroll
+    for (int q = 0; q < kVecs; ++q)
+      if (v0 + 32 * q < row_vecs) dst[v0 + 32 * q] = a[q];
+  }
+}
+
+// xp non-null: the CTA also gathers the dispatched rows (one warp per row),
+// which saves the gather launch for the smallest batches.
 __global__ void __launch_bounds__(1024) dispatch_small(const int32_t* __restrict__ idx, int TK,
                                                        int E, int T, int has_shared,
                                                        int32_t* __restrict__ counts,
                                                        int32_t* __restrict__ offsets,
                                                        int32_t* __restrict__ perm,
                                                        int32_t* __restrict__ inv, TileSpec ts,
-                                                       WsHeader* __restrict__ hdr) {
+                                                       WsHeader* __restrict__ hdr,
+                                                       const uint4* __restrict__ x, int K,
+                                                       int row_vecs, uint4* __restrict__ xp) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int dyn_smem[];
   dispatch_block(idx, TK, E, T, has_shared, counts, offsets, perm, inv, ts, hdr, dyn_smem);
+  if (xp == nullptr) return;
+  __syncthreads();   // every warp's perm rows are written and visible to the CTA
+  // The rows' vectors spread over all threads, a few loads in flight each
+  // (the CTA's 64 registers per thread leave no room for a warp per row).
+  constexpr int kVecs = 4;
+  const int total = TK * row_vecs;
+  for (int i0 = threadIdx.x; i0 < total; i0 += kVecs * blockDim.x) {
+    uint4 a[kVecs];
+    int dst[kVecs];
+#pragma unroll
+    for (int q = 0; q < kVecs; ++q) {
+      const int i = i0 + q * blockDim.x;
+      dst[q] = -1;
+      if (i < total) {
+        const int row = i / row_vecs, v = i - row * row_vecs;
+        const int c = perm[row];
+        if ((unsigned)c < (unsigned)TK) {   // else: a rejected copy, reported in the status
+          a[q] = x[(size_t)(c / K) * row_vecs + v];
+          dst[q] = i;
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kVecs; ++q)
+      if (dst[q] >= 0) xp[dst[q]] = a[q];
+  }
 }
 
-// Gather of dispatched activation rows: xp[row] = x[perm[row] / K] (bf16,
-// 16-byte vectors), so the tensor-core GEMM reads contiguous rows. One warp
-// per row; each lane issues up to 16 vector loads before its first store
-// (a 4096-wide row in one memory round trip).
+// Gather of dispatched activation rows, so the tensor-core GEMM reads
+// contiguous rows: one warp per row.
 __global__ void __launch_bounds__(256) gather_rows(const uint4* __restrict__ x,
                                                    const int32_t* __restrict__ perm, int TK,
                                                    int K, int row_vecs, uint4* __restrict__ xp) {
   pdl_wait();
   pdl_trigger();
-  constexpr int kVecs = 16;   // vectors in flight per lane
-  const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
-  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < TK; row += warps) {
-    const uint4* src = x + (size_t)(perm[row] / K) * row_vecs;
-    uint4* dst = xp + (size_t)row * row_vecs;
-    for (int v0 = lane; v0 < row_vecs; v0 += 32 * kVecs) {
-      uint4 a[kVecs];
-#pragma unroll
-      for (int q = 0; q < kVecs; ++q)
-        if (v0 + 32 * q < row_vecs) a[q] = src[v0 + 32 * q];
-#pragma unroll
-      for (int q = 0; q < kVecs; ++q)
-        if (v0 + 32 * q < row_vecs) dst[v0 + 32 * q] = a[q];
-    }
-  }
+  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < TK; row += warps)
+    gather_row(x, perm, TK, K, row_vecs, xp, row, threadIdx.x & 31);
 }
 
 static TileSpec make_tile_spec(const moe_layer_desc& d, const WsLayout& L, char* ws,
@@ -511,11 +553,15 @@ static TileSpec make_tile_spec(const moe_layer_desc& d, const WsLayout& L, char*
   return ts;
 }
 
-cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws,
-                            const int32_t* idx, int32_t* counts, int32_t* offsets,
-                            int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st,
-                            bool shared_tiles) {
+// Dispatch; with x and xp (bf16 layers) also the gather of the dispatched
+// rows into xp, inside the one-CTA dispatch for batches of at most
+// kFusedGatherCopies copies, else as its own launch after the dispatch.
+static cudaError_t dispatch_impl(const moe_layer_desc& d, const WsLayout& L, char* ws,
+                                 const int32_t* idx, int32_t* counts, int32_t* offsets,
+                                 int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st,
+                                 bool shared_tiles, const void* x, void* xp, int num_sms) {
   const int TK = d.T * d.K;
+  const bool fuse_gather = xp != nullptr && TK <= kFusedGatherCopies;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
   int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
@@ -537,8 +583,12 @@ cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws
       if (e != cudaSuccess) return e;
       if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
     }
-    return launch_pdl(dispatch_small, dim3(1), dim3(threads), smem, st, idx, TK, d.E, d.T,
-                      has_shared, counts, offsets, perm, inv, ts, hdr);
+    e = launch_pdl(dispatch_small, dim3(1), dim3(threads), smem, st, idx, TK, d.E, d.T,
+                   has_shared, counts, offsets, perm, inv, ts, hdr,
+                   static_cast<const uint4*>(fuse_gather ? x : nullptr), d.K, d.H * 2 / 16,
+                   static_cast<uint4*>(fuse_gather ? xp : nullptr));
+    if (e != cudaSuccess || fuse_gather || xp == nullptr) return e;
+    return launch_gather_rows(d, x, perm, xp, num_sms, st);
   }
   cudaError_t e = cudaSuccess;
   if (TK > 0)
@@ -553,7 +603,24 @@ cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws
   if (TK > 0)
     e = launch_pdl(chunk_scatter, dim3(n_chunks), dim3(256), 0, st, idx, TK, d.E,
                    (const int32_t*)base, perm, inv);
-  return e;
+  if (e != cudaSuccess || xp == nullptr) return e;
+  return launch_gather_rows(d, x, perm, xp, num_sms, st);
+}
+
+cudaError_t launch_dispatch(const moe_layer_desc& d, const WsLayout& L, char* ws,
+                            const int32_t* idx, int32_t* counts, int32_t* offsets,
+                            int32_t* perm, int32_t* inv, bool tc_tiles, cudaStream_t st,
+                            bool shared_tiles) {
+  return dispatch_impl(d, L, ws, idx, counts, offsets, perm, inv, tc_tiles, st, shared_tiles,
+                       nullptr, nullptr, 0);
+}
+
+cudaError_t launch_dispatch_gather(const moe_layer_desc& d, const WsLayout& L, char* ws,
+                                   const int32_t* idx, int32_t* counts, int32_t* offsets,
+                                   int32_t* perm, int32_t* inv, cudaStream_t st,
+                                   bool shared_tiles, const void* x, void* xp, int num_sms) {
+  return dispatch_impl(d, L, ws, idx, counts, offsets, perm, inv, /*tc_tiles=*/true, st,
+                       shared_tiles, x, xp, num_sms);
 }
 
 // The same three dispatch kernels with caller-provided scratch: hist and base
