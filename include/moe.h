@@ -163,7 +163,10 @@ moe_status moe_topk_from_logits_noisy(const moe_layer_desc* desc, const float* l
  * "Kimi K3 专家路由不均衡诊断" §三 (np.add.at counts) and §五 (no dropping).
  *   topk_idx [T, K] int32 in [0, E) (input);
  *   counts [E], offsets [E + 1], perm [T*K], inv [T*K] int32 outputs:
- *   copy c = t*K + k lands in row inv[c]; perm[row] = c. */
+ *   copy c = t*K + k lands in row inv[c]; perm[row] = c.
+ * A copy whose index is outside [0, E) is skipped (counts then sum to less
+ * than T*K, and its perm / inv entries are not written); the workspace
+ * status word records it, and moe_check_status reports MOE_ERR_INVALID_ARG. */
 moe_status moe_dispatch(const moe_layer_desc* desc, const int32_t* topk_idx, int32_t* counts,
                         int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
                         size_t ws_bytes, moe_stream stream);
@@ -266,7 +269,9 @@ moe_status moe_bias_update(const moe_layer_desc* desc, const int32_t* counts, fl
                            float gamma, moe_stream stream);
 
 /* Reads and clears the workspace status word (synchronises `stream`):
- * MOE_OK, or MOE_ERR_TIMEOUT if a bounded device wait ran out. */
+ * MOE_OK; MOE_ERR_TIMEOUT if a bounded device wait ran out (this takes
+ * precedence); MOE_ERR_INVALID_ARG if a dispatch met a top-K index outside
+ * [0, E). */
 moe_status moe_check_status(void* ws, size_t ws_bytes, moe_stream stream);
 
 /* Static description of a status code. */
