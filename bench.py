@@ -53,6 +53,8 @@ def parse_args():
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--sweep-all", action="store_true", help="also measure every other workload point")
+    p.add_argument("--cold-l2", action="store_true",
+                   help="sweep points also report the median forward with L2 flushed before each call")
     return p.parse_args()
 
 
@@ -421,6 +423,27 @@ class Runner:
         del g
         return start.elapsed_time(end)
 
+    def timed_cold(self, iters, warmup=3):
+        """Median forward time (ms) with L2 flushed before every call: a buffer
+        of twice the L2 size is written between calls, outside the events
+        around the forward (both on the current stream)."""
+        props = torch.cuda.get_device_properties(torch.cuda.current_device())
+        l2 = int(getattr(props, "L2_cache_size", 0)) or (126 << 20)
+        flush = torch.empty(2 * l2, dtype=torch.uint8, device="cuda")
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(iters)]
+        for i in range(warmup + iters):
+            flush.fill_(i & 0xFF)
+            if i >= warmup:
+                evs[i - warmup][0].record()
+            self.step()
+            if i >= warmup:
+                evs[i - warmup][1].record()
+        torch.cuda.synchronize()
+        times = sorted(a.elapsed_time(b) for a, b in evs)
+        del flush
+        return times[len(times) // 2]
+
     def stages(self, steps):
         """Per-stage device times (ms, mean over steps) from events recorded
         between the kernels of moe_layer_forward_profiled."""
@@ -557,7 +580,7 @@ def run_ours(args, wl, T):
         "clocks": clocks,
     }
     if not args.no_sweep and world == 1:
-        line["sweep"] = sweep(M, wl, dev, T, peaks, args.sweep_all)
+        line["sweep"] = sweep(M, wl, dev, T, peaks, args.sweep_all, args.cold_l2)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, host, R.x_host, T)
     if rank == 0:
@@ -567,7 +590,7 @@ def run_ours(args, wl, T):
         dist.destroy_process_group()
 
 
-def measure_point(M, wl, dev, T, peaks, steps=20, warmup=5):
+def measure_point(M, wl, dev, T, peaks, steps=20, warmup=5, cold=False):
     R = Runner(M, wl, dev, T, replica=0)
     ms, _ = R.timed(steps, warmup, 1, None)
     st = R.stages(steps)
@@ -575,14 +598,19 @@ def measure_point(M, wl, dev, T, peaks, steps=20, warmup=5):
     bound, t_roof = roofline_bound(alg["flops"], alg["bytes"], peaks)
     ms_step = ms / steps
     graph_ms = R.timed_graph(steps, warmup) / steps
-    return {"workload": wl.key, "T": T, "tokens_per_s": T / (ms_step / 1e3), "us_per_step": 1e3 * ms_step,
-            "graph_us_per_step": 1e3 * graph_ms, "graph_frac": 1e3 * t_roof / graph_ms,
-            "bound": bound, "roofline_us": 1e6 * t_roof, "frac": 1e3 * t_roof / ms_step,
-            "experts_touched": R.touched(), "stages_us": {k: 1e3 * v for k, v in st.items()}}
+    out = {"workload": wl.key, "T": T, "tokens_per_s": T / (ms_step / 1e3), "us_per_step": 1e3 * ms_step,
+           "graph_us_per_step": 1e3 * graph_ms, "graph_frac": 1e3 * t_roof / graph_ms,
+           "bound": bound, "roofline_us": 1e6 * t_roof, "frac": 1e3 * t_roof / ms_step,
+           "experts_touched": R.touched(), "stages_us": {k: 1e3 * v for k, v in st.items()}}
+    if cold:
+        cold_ms = R.timed_cold(max(steps, 50))
+        out["cold_l2_us_per_step"] = 1e3 * cold_ms
+        out["cold_l2_frac"] = 1e3 * t_roof / cold_ms
+    return out
 
 
-def sweep(M, wl, dev, T_main, peaks, all_workloads):
-    out = [measure_point(M, wl, dev, T, peaks) for T in wl.Ts if T != T_main]
+def sweep(M, wl, dev, T_main, peaks, all_workloads, cold=False):
+    out = [measure_point(M, wl, dev, T, peaks, cold=cold) for T in wl.Ts if T != T_main]
     if all_workloads:
         for key in ("c3", "c4", "c5", "c1"):
             if key == wl.key:
@@ -591,7 +619,7 @@ def sweep(M, wl, dev, T_main, peaks, all_workloads):
             host = mi.draw_layer(w2)
             d2 = {k: (v.cuda() if v is not None else None) for k, v in host.items()}
             for T in w2.Ts:
-                out.append(measure_point(M, w2, d2, T, peaks))
+                out.append(measure_point(M, w2, d2, T, peaks, cold=cold))
             del d2
             torch.cuda.empty_cache()
     return out
