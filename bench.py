@@ -202,7 +202,9 @@ class ClockSampler:
         except Exception:
             self.thread = None
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            scratch = os.path.join(ROOT, "_build")
+            os.makedirs(scratch, exist_ok=True)
+            fd, self.path = tempfile.mkstemp(suffix=".csv", dir=scratch)
             os.close(fd)
             idx = self.device.index if self.device.index is not None else 0
             self.proc = subprocess.Popen(

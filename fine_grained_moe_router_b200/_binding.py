@@ -46,7 +46,7 @@ class MoEStats(ctypes.Structure):
                 ("capacity", ctypes.c_int32), ("max_load", ctypes.c_int32),
                 ("min_load", ctypes.c_int32), ("num_stragglers", ctypes.c_int32),
                 ("skew_ratio", ctypes.c_double), ("gini", ctypes.c_double),
-                ("overflow_rate", ctypes.c_double)]
+                ("overflow_rate", ctypes.c_double), ("max_over_mean", ctypes.c_double)]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}

@@ -53,6 +53,10 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     if not force and not _stale():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
+    # the compiler's intermediate files stay inside the repository too
+    tmp = os.path.join(BUILD, "tmp")
+    os.makedirs(tmp, exist_ok=True)
+    env = dict(os.environ, TMPDIR=tmp)
     cc = nvcc()
     objs = []
 
@@ -61,7 +65,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         cmd = [cc, *ARCH, *FLAGS, *extra_flags, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
-        r = subprocess.run(cmd, capture_output=True, text=True)
+        r = subprocess.run(cmd, capture_output=True, text=True, env=env)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
         if verbose and (r.stdout or r.stderr):
@@ -74,7 +78,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     cmd = [cc, *ARCH, "-shared", "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
-    r = subprocess.run(cmd, capture_output=True, text=True)
+    r = subprocess.run(cmd, capture_output=True, text=True, env=env)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)

@@ -195,6 +195,7 @@ __global__ void __launch_bounds__(512) expert_stats_kernel(const int32_t* __rest
     const long long n = E;
     s.gini = (S == 0) ? 0.0 : (double)(2 * R - (n + 1) * S) / (double)(n * S);
     s.overflow_rate = (TK == 0) ? 0.0 : (double)over / (double)TK;
+    s.max_over_mean = (TK == 0) ? 0.0 : (double)mx * (double)n / (double)TK;
     *out = s;
   }
 }

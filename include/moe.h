@@ -121,6 +121,7 @@ typedef struct {
   double skew_ratio;        /* max_load / (min_load + 1e-5) */
   double gini;              /* (2*sum_i i*c_(i) - (n+1)*S) / (n*S), 0 if S = 0 */
   double overflow_rate;     /* overflow / (T*K), 0 if T*K = 0 */
+  double max_over_mean;     /* max_load / (T*K / E), 0 if T*K = 0 */
 } moe_stats;
 
 /* Bytes of workspace every call below needs for this shape (one size for

@@ -355,6 +355,9 @@ def load_stats(counts: np.ndarray, T: int, K: int, cf_num: int = 5, cf_den: int 
         "gini": gini_exact(c),
         "overflow": overflow,
         "overflow_rate": float(overflow) / float(T * K) if T * K else 0.0,
+        # hottest expert over the mean load T*K/E: the skew that stays finite
+        # when an expert is idle (max/(min + 1e-5) is then 1e5 * max)
+        "max_over_mean": float(mx) * float(E) / float(T * K) if T * K else 0.0,
         "num_stragglers": int(np.count_nonzero(c > cap)),
         "straggler_mask": (c > cap).astype(np.uint8),
     }

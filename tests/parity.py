@@ -107,7 +107,7 @@ def check_dispatch_valid(idx, counts, offsets, perm, inv, E):
 def stats_equal(got: dict, want: dict):
     for k in ("num_copies", "capacity", "max_load", "min_load", "overflow", "num_stragglers"):
         assert int(got[k]) == int(want[k]), k
-    for k in ("skew_ratio", "gini", "overflow_rate"):
+    for k in ("skew_ratio", "gini", "overflow_rate", "max_over_mean"):
         assert got[k] == want[k], (k, got[k], want[k])     # bit-exact: same exact formula
 
 

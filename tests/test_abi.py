@@ -11,6 +11,12 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moe.h")
+SCRATCH = os.path.join(ROOT, "_build", "tests")   # compiled probes stay inside the repository
+
+
+def _tmpdir():
+    os.makedirs(SCRATCH, exist_ok=True)
+    return tempfile.TemporaryDirectory(dir=SCRATCH)
 
 
 @pytest.fixture(scope="module")
@@ -52,33 +58,36 @@ def test_struct_layout_matches_header(M):
 int main(void) {
   printf("%zu %zu %zu %zu\n", sizeof(moe_layer_desc), sizeof(moe_layer_weights),
          sizeof(moe_routing), sizeof(moe_stats));
-  printf("%zu %zu %zu %zu %zu\n", offsetof(moe_stats, capacity), offsetof(moe_stats, num_stragglers),
-         offsetof(moe_stats, skew_ratio), offsetof(moe_stats, gini), offsetof(moe_stats, overflow_rate));
+  printf("%zu %zu %zu %zu %zu %zu\n", offsetof(moe_stats, capacity), offsetof(moe_stats, num_stragglers),
+         offsetof(moe_stats, skew_ratio), offsetof(moe_stats, gini), offsetof(moe_stats, overflow_rate),
+         offsetof(moe_stats, max_over_mean));
   printf("%zu %zu\n", offsetof(moe_layer_desc, dtype), offsetof(moe_routing, logits));
   return 0;
 }
 '''
-    with tempfile.TemporaryDirectory() as d:
+    with _tmpdir() as d:
         c = os.path.join(d, "layout.c")
         exe = os.path.join(d, "layout")
         open(c, "w").write(prog)
-        subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
+        subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True,
+                       env=dict(os.environ, TMPDIR=d))
         got = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()
     got = [int(v) for v in got]
     want = [ctypes.sizeof(M.MoELayerDesc), ctypes.sizeof(M.MoELayerWeights), ctypes.sizeof(M.MoERouting),
             ctypes.sizeof(M.MoEStats),
             M.MoEStats.capacity.offset, M.MoEStats.num_stragglers.offset, M.MoEStats.skew_ratio.offset,
-            M.MoEStats.gini.offset, M.MoEStats.overflow_rate.offset,
+            M.MoEStats.gini.offset, M.MoEStats.overflow_rate.offset, M.MoEStats.max_over_mean.offset,
             M.MoELayerDesc.dtype.offset, M.MoERouting.logits.offset]
     assert got == want
 
 
 def test_header_compiles_as_c_and_cxx():
-    with tempfile.TemporaryDirectory() as d:
+    with _tmpdir() as d:
         for lang, cc in (("c", "gcc"), ("cpp", "g++")):
             f = os.path.join(d, "inc." + lang)
             open(f, "w").write('#include "moe.h"\nint main(void){return (int)MOE_OK;}\n')
-            subprocess.run([cc, "-Wall", "-Werror", "-I", os.path.dirname(HEADER), f, "-o", f + ".out"], check=True)
+            subprocess.run([cc, "-Wall", "-Werror", "-I", os.path.dirname(HEADER), f, "-o", f + ".out"], check=True,
+                           env=dict(os.environ, TMPDIR=d))
 
 
 def test_workspace_size_rejects_bad_descriptors(M):

@@ -150,6 +150,13 @@ def _stats_skew_without_epsilon(counts, T, K, cf_num=5, cf_den=4):
     return st
 
 
+def _stats_max_over_mean_of_min(counts, T, K, cf_num=5, cf_den=4):
+    st = _orig["load_stats"](counts, T, K, cf_num, cf_den)
+    c = np.asarray(counts, np.int64)
+    st["max_over_mean"] = float(c.min()) * c.size / (T * K) if T * K else 0.0
+    return st
+
+
 MUTANTS = {
     "ties_to_higher_index": ("select_topk", _topk_high_index_ties),
     "weights_not_renormalised": ("select_topk", _topk_no_renorm),
@@ -172,6 +179,7 @@ MUTANTS = {
     "offsets_inclusive": ("expert_offsets", _offsets_inclusive),
     "combine_unweighted": ("combine", _combine_unweighted),
     "skew_without_epsilon": ("load_stats", _stats_skew_without_epsilon),
+    "max_over_mean_of_min": ("load_stats", _stats_max_over_mean_of_min),
 }
 
 PIN_TESTS = [
@@ -194,6 +202,7 @@ PIN_TESTS = [
     pins.test_gumbel_max_picks_each_expert_with_its_softmax_probability,
     pins.test_noisy_weights_are_the_softmax_of_the_noisy_scores,
     pins.test_combine_worked_example,
+    pins.test_max_over_mean_closed_forms,
     pins.test_stagewise_grouped_ffn_and_combine_equal_layer_definition,
     pins.test_bias_update_moves_only_overloaded_and_idle_experts,
     pins.test_bias_update_is_a_fixed_point_for_an_even_load,

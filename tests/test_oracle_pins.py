@@ -315,6 +315,15 @@ def test_gini_matches_mean_absolute_difference_form():
         assert oracle.gini_exact(one_hot) == pytest.approx((n - 1) / n, abs=1e-15)
 
 
+def test_max_over_mean_closed_forms():
+    """Hottest expert over the mean load T*K/E: 1 for an even load, E when a
+    single copy exists, and a hand-worked uneven case."""
+    assert oracle.load_stats(np.full(8, 5), 20, 2)["max_over_mean"] == 1.0
+    assert oracle.load_stats(np.eye(1, 16, 3, dtype=np.int64)[0], 1, 1)["max_over_mean"] == 16.0
+    assert oracle.load_stats(np.array([1, 2, 3, 4]), 5, 2)["max_over_mean"] == 1.6   # 4 / (10/4)
+    assert oracle.load_stats(np.zeros(4, np.int64), 0, 2)["max_over_mean"] == 0.0
+
+
 def test_load_stats_golden_cases():
     for case in _golden()["stats"]:
         T, K = case["T"], case["K"]
