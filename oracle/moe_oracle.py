@@ -236,7 +236,8 @@ def combine(y_rows, w, inv, y_shared=None):
 # --------------------------------------------------------------------------
 # a9  full layer: route, dispatch, experts, weighted combine (+ shared)
 # --------------------------------------------------------------------------
-def moe_layer_forward(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None, noise=None):
+def moe_layer_forward(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None, noise=None,
+                      logits=None):
     """Forward pass of one fine-grained MoE FFN layer.
 
     Steps: gate logits, Softmax(l + B) selection of the top K with
@@ -253,6 +254,11 @@ def moe_layer_forward(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None, noise
     those tokens only (routing and dispatch always cover all T tokens).
     ``noise``: optional [T, E] Gumbel draws for noisy routing ([MOE-ARCH]
     §2.3; see ``selection_scores``).
+    ``logits``: optional [T, E] gate logits given by the caller (for example
+    the fp32 logits a GPU run produced); the selection is then taken on
+    these instead of on ``x @ W_r^T``, and every later step is unchanged. A
+    parity check routes the oracle this way, so that both sides decide the
+    top-K on the same fp32 numbers.
 
     Returns dict with logits, idx, w, s, counts, offsets, perm, inv and
     ``y`` [len(tokens), H] float64.
@@ -260,7 +266,12 @@ def moe_layer_forward(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None, noise
     x = np.asarray(x, dtype=np.float64)
     T, H = x.shape
     E = np.asarray(w_router).shape[0]
-    logits = router_logits(x, w_router)
+    if logits is None:
+        logits = router_logits(x, w_router)
+    else:
+        logits = np.asarray(logits, dtype=np.float64)
+        if logits.shape != (T, E):
+            raise ValueError("given logits must have shape [T, E]")
     idx, w, s = select_topk(logits, bias, K, noise)
     counts, off, perm, inv = dispatch(idx, E)
 

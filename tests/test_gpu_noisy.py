@@ -7,7 +7,7 @@ import torch
 
 import moe_inputs as mi
 import oracle
-from parity import DeviceLayer, W_TOL, compare_routing, rel_max_err, to_np, y_tol
+from parity import DeviceLayer, W_TOL, check_layer, routing_buffers, routing_np, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -40,19 +40,6 @@ def test_noisy_topk_from_logits_bit_exact(M, T, E, K, ties):
     assert np.max(np.abs(to_np(w) - ref_w)) <= W_TOL
 
 
-def _routing(wl, T):
-    E, K = wl.E, wl.K
-    return {
-        "topk_idx": torch.empty((T, K), dtype=torch.int32, device="cuda"),
-        "topk_w": torch.empty((T, K), dtype=torch.float32, device="cuda"),
-        "counts": torch.empty(E, dtype=torch.int32, device="cuda"),
-        "offsets": torch.empty(E + 1, dtype=torch.int32, device="cuda"),
-        "perm": torch.empty(T * K, dtype=torch.int32, device="cuda"),
-        "inv": torch.empty(T * K, dtype=torch.int32, device="cuda"),
-        "logits": torch.empty((T, E), dtype=torch.float32, device="cuda"),
-    }
-
-
 @pytest.mark.parametrize("key,shape,T", [("c3", dict(H=512, D=256, Ds=512), 16),
                                          ("c4", dict(H=512, D=256, Ds=512), 200),
                                          ("c1", {}, 64)])
@@ -64,21 +51,14 @@ def test_noisy_layer_matches_oracle(M, key, shape, T):
     g = mi.draw_gumbel(T, wl.E, seed=wl.seed + T)
     xd = x.cuda()
     y = torch.full_like(xd, float("nan"))
-    r = _routing(wl, T)
+    r = routing_buffers(wl, T)
     ws = M.alloc_workspace(d)
     M.moe_layer_forward_noisy(d, L.weights(M), xd, g.cuda(), y, M.make_routing(**r), ws)
     torch.cuda.synchronize()
     assert M.moe_check_status(ws) == 0
     gn = g.numpy()
-    ref = oracle.moe_layer_forward(mi.to_f64(x), L.wr64, L.bias, L.w1_64, L.w2_64, L.ws1_64,
-                                   L.ws2_64, wl.K, noise=gn)
-    uniq, _, _ = compare_routing(wl, to_np(r["logits"]), to_np(r["topk_idx"]), to_np(r["topk_w"]),
-                                 ref["logits"], L.bias, noise=gn)
-    if uniq.all():
-        for k in ("counts", "offsets", "perm", "inv"):
-            assert (to_np(r[k]) == ref[k]).all(), k
-    err = rel_max_err(to_np(y)[uniq], ref["y"][uniq])
-    assert err <= y_tol(wl), f"max |y - y_ref| = {err:.3e} x RMS"
+    # the oracle is routed from the GPU's logits with the same noise
+    ref = check_layer(wl, x, L, routing_np(r), to_np(y), noise=gn)
     # the noise changes the routing of some tokens
     plain_idx, _, _ = oracle.select_topk(ref["logits"], L.bias, wl.K)
     assert (plain_idx != ref["idx"]).any()

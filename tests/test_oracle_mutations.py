@@ -103,8 +103,15 @@ def _ffn_transposed_second(rows, w1, w2):
     return h @ w2.T * 1.0001
 
 
-def _layer_no_shared(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None, noise=None):
-    return _orig["moe_layer_forward"](x, w_router, bias, w1, w2, None, None, K, tokens, noise)
+def _layer_no_shared(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None, noise=None,
+                     logits=None):
+    return _orig["moe_layer_forward"](x, w_router, bias, w1, w2, None, None, K, tokens, noise,
+                                      logits)
+
+
+def _layer_ignores_given_logits(x, w_router, bias, w1, w2, ws1, ws2, K, tokens=None, noise=None,
+                                logits=None):
+    return _orig["moe_layer_forward"](x, w_router, bias, w1, w2, ws1, ws2, K, tokens, noise)
 
 
 def _stats_overflow_counts_experts(counts, T, K, cf_num=5, cf_den=4):
@@ -170,6 +177,7 @@ MUTANTS = {
     "ffn_without_gelu": ("expert_ffn", _ffn_no_gelu),
     "ffn_second_linear_transposed": ("expert_ffn", _ffn_transposed_second),
     "shared_expert_dropped": ("moe_layer_forward", _layer_no_shared),
+    "given_logits_ignored": ("moe_layer_forward", _layer_ignores_given_logits),
     "overflow_counts_experts": ("load_stats", _stats_overflow_counts_experts),
     "gumbel_noise_ignored": ("selection_scores", _scores_ignore_noise),
     "noisy_weights_from_clean_scores": ("select_topk", _topk_weights_from_clean_scores),
@@ -195,6 +203,7 @@ PIN_TESTS = [
     lambda: pins.test_identical_experts_give_single_ffn_for_any_routing(2),
     pins.test_K1_is_an_identity_scatter_of_the_chosen_expert,
     pins.test_layer_sum_over_k_matches_explicit_per_token_loop,
+    pins.test_given_logits_decide_the_routing,
     pins.test_gini_golden_cases,
     pins.test_gini_matches_mean_absolute_difference_form,
     pins.test_load_stats_golden_cases,

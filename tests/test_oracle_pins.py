@@ -243,6 +243,35 @@ def test_K1_is_an_identity_scatter_of_the_chosen_expert():
                                    rtol=1e-12, atol=1e-13)
 
 
+def test_given_logits_decide_the_routing():
+    """With caller-given logits the selection follows them, not x W_r^T: a
+    one-hot logit row sends every token to its expert (K=1 gives exactly that
+    expert's FFN), and with K=2 the weights are the renormalised softmax of
+    the two given scores (closed form 1/(1+e^-d))."""
+    rng = _rng(26)
+    T, H, E, D = 23, 16, 6, 20
+    x, wr, w1, w2, _, _ = _rand_layer(rng, T, H, E, D)
+    hot = rng.integers(0, E, size=T)
+    lg = np.full((T, E), -3.0)
+    lg[np.arange(T), hot] = 2.0
+    out = oracle.moe_layer_forward(x, wr, None, w1, w2, None, None, 1, logits=lg)
+    assert (out["idx"][:, 0] == hot).all()
+    assert (out["counts"] == np.bincount(hot, minlength=E)).all()
+    for t in range(T):
+        np.testing.assert_allclose(out["y"][t], _torch_ffn(x[t:t + 1], w1[hot[t]], w2[hot[t]])[0],
+                                   rtol=1e-12, atol=1e-13)
+    # K = 2: second-best score 2.0 - d on the next expert (cyclically)
+    d = 0.75
+    lg2 = lg.copy()
+    lg2[np.arange(T), (hot + 1) % E] = 2.0 - d
+    out2 = oracle.moe_layer_forward(x, wr, None, w1, w2, None, None, 2, logits=lg2)
+    assert (out2["idx"][:, 0] == hot).all() and (out2["idx"][:, 1] == (hot + 1) % E).all()
+    np.testing.assert_allclose(out2["w"][:, 0], 1.0 / (1.0 + math.exp(-d)), rtol=1e-7)
+    # the router's own logits route differently on this input
+    own = oracle.moe_layer_forward(x, wr, None, w1, w2, None, None, 1)
+    assert (own["idx"][:, 0] != hot).any()
+
+
 def test_layer_sum_over_k_matches_explicit_per_token_loop():
     """y[t] = sum_k w[t,k] * FFN_{idx[t,k]}(x[t]) (+ shared), token by token."""
     rng = _rng(24)
