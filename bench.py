@@ -86,7 +86,7 @@ def algorithmic(wl, T, touched, counts=None):
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the two
 # expert-GEMM launches of one step, from one ncu capture of this workload
-# (profiles/grouped_gemm_tc_mixtral_T4096.md). Valid only for the kernel code
+# (the committed ncu summary of the expert GEMM). Valid only for the kernel code
 # it was measured on: the key is a fingerprint of the GEMM source and the
 # headers it includes with comments and whitespace removed, so any change to
 # the code (not to its comments) makes it null.

@@ -589,14 +589,30 @@ static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer
   // the router and dispatch need.
   SideStream* side = nullptr;
   std::unique_lock<std::mutex> side_lock;
+  // Once the side stream has forked from `st`, every return joins it back:
+  // an error after the fork must not leave the shared expert's launches
+  // running unjoined (that would also invalidate a graph capture).
+  struct SideJoin {
+    SideStream* side = nullptr;
+    cudaStream_t st = nullptr;
+    bool recorded = false;
+    ~SideJoin() {
+      if (!side) return;
+      if (!recorded) cudaEventRecord(side->join, side->stream);
+      cudaStreamWaitEvent(st, side->join, 0);
+    }
+  } join_guard;
   if (tc && d.Ds > 0 && !L.sp.pair && d.T >= kSideStreamMinT) {
     side = side_stream();
     if (!side) return MOE_ERR_CUDA;
     side_lock = std::unique_lock<std::mutex>(side->mu);
     MOE_CUDA_TRY(cudaEventRecord(side->fork, st));
     MOE_CUDA_TRY(cudaStreamWaitEvent(side->stream, side->fork, 0));
+    join_guard.side = side;
+    join_guard.st = st;
     MOE_TRY(run_shared_ffn(d, L, w, x, W.ws1, W.ws2, side->stream));
     MOE_CUDA_TRY(cudaEventRecord(side->join, side->stream));
+    join_guard.recorded = true;
   }
   MOE_CUDA_TRY(mark(0));
   MOE_TRY(run_router(d, L, w, x, W.w_router, W.expert_bias, idx, tw, R.logits, st, noise));
@@ -612,7 +628,10 @@ static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer
   MOE_TRY(run_grouped_ffn(d, L, w, x, perm, W.w1, W.w2, W.ws1, W.ws2, yr, ys, st,
                           /*split=*/true, ev ? ev + 3 : nullptr, /*with_shared=*/side == nullptr));
   MOE_CUDA_TRY(mark(4));
-  if (side) MOE_CUDA_TRY(cudaStreamWaitEvent(st, side->join, 0));
+  if (side) {
+    join_guard.side = nullptr;   // joined here
+    MOE_CUDA_TRY(cudaStreamWaitEvent(st, side->join, 0));
+  }
   MOE_CUDA_TRY(launch_combine(d, yr, tw, inv, ys, y, st, L.sp.gemm2_routed, L.sp.gemm2_shared));
   MOE_CUDA_TRY(mark(5));
   return MOE_OK;

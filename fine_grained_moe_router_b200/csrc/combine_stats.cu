@@ -94,8 +94,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   float acc[V::N];
 #pragma unroll
   for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
+  const unsigned TK = (unsigned)T_ * (unsigned)K;
   for (int k = 0; k < K; ++k) {
     const int row = inv[(size_t)t * K + k];
+    // a copy the dispatch could not place (inv = -1, reported in the
+    // workspace status) contributes nothing
+    if ((unsigned)row >= TK) continue;
     const float wk = w[(size_t)t * K + k];
     const float* src = y_rows + (size_t)row * H + h;
 #pragma unroll

@@ -6,13 +6,19 @@
 // the expert and scattered back. "Kimi K3 专家路由不均衡诊断" §三 counts hits
 // per expert; §五 forbids dropping copies, so every copy gets a row.
 //
-// Three kernels, no global atomics:
-//   1. chunk_histogram   per-chunk expert counts (shared-memory counters)
+// Three kernels, no atomics in the counting or the placement:
+//   1. chunk_histogram   per-chunk expert counts: each warp counts its own
+//                        range of copies into a private row of counters (the
+//                        lanes holding one expert find each other with
+//                        __match_any_sync and the lowest adds the group's size)
 //   2. scan_and_tiles    one CTA: counts, exclusive offsets, per-(chunk,
 //                        expert) bases, and the grouped-GEMM tile lists
 //   3. chunk_scatter     stable placement: inside a chunk, warps own
 //                        consecutive copy ranges and rank equal experts with
 //                        __match_any_sync, so the order is ascending copy id.
+// A copy whose expert index is outside [0, E) is not placed: its inv entry
+// is -1, the rows past the placed copies hold perm = -1, and the status word
+// records kStatusBadIndex.
 // Batches of at most one chunk (kChunk copies) run all three steps in one CTA
 // (dispatch_small). gather_rows then copies the dispatched activation rows
 // for the tensor-core GEMMs; for the smallest batches (kFusedGatherCopies)
@@ -26,27 +32,52 @@
 
 namespace moe {
 
-__global__ void __launch_bounds__(256) chunk_histogram(const int32_t* __restrict__ idx, int TK,
-                                                       int E, int32_t* __restrict__ hist,
-                                                       uint32_t* __restrict__ status) {
+// Counts the copies [w0, w1) by expert into the warp's own counter row
+// cnt_row[0..E) without atomics: in each round of 32 copies the lanes that
+// hold the same expert find each other with __match_any_sync and the lowest
+// of them adds the group's size, so no two lanes write one counter at once.
+// Returns true (on every lane) if some copy's expert is outside [0, E).
+__device__ __forceinline__ bool warp_count(const int32_t* __restrict__ idx, int w0, int w1, int E,
+                                           int* cnt_row) {
+  const int lane = threadIdx.x & 31;
+  const unsigned below = (1u << lane) - 1u;
+  bool bad = false;
+  for (int i0 = w0; i0 < w1; i0 += 32) {
+    const int i = i0 + lane;
+    const bool live = i < w1;
+    const int e = live ? idx[i] : -1;
+    const bool ok = live && (unsigned)e < (unsigned)E;
+    bad |= live && !ok;
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+    if (ok && (peers & below) == 0) cnt_row[e] += __popc(peers);
+    __syncwarp();
+  }
+  return __any_sync(0xffffffffu, bad);
+}
+
+constexpr int kHistWarps = 8;
+
+__global__ void __launch_bounds__(kHistWarps * 32) chunk_histogram(const int32_t* __restrict__ idx,
+                                                                  int TK, int E,
+                                                                  int32_t* __restrict__ hist,
+                                                                  uint32_t* __restrict__ status) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int h[kMaxE];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+  __shared__ int cnt[kHistWarps][kMaxE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kHistWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
   __syncthreads();
   const int c0 = blockIdx.x * kChunk;
-  const int c1 = min(TK, c0 + kChunk);
-  bool bad = false;
-  for (int i = c0 + threadIdx.x; i < c1; i += blockDim.x) {
-    const int e = idx[i];
-    if ((unsigned)e < (unsigned)E)
-      atomicAdd(&h[e], 1);
-    else
-      bad = true;
-  }
-  if (bad) atomicOr(status, kStatusBadIndex);
+  const int per_warp = kChunk / kHistWarps;
+  const int w0 = min(TK, c0 + warp * per_warp), w1 = min(TK, w0 + per_warp);
+  if (warp_count(idx, w0, w1, E, cnt[warp]) && lane == 0) atomicOr(status, kStatusBadIndex);
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)blockIdx.x * E + e] = h[e];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kHistWarps; ++w) c += cnt[w][e];
+    hist[(size_t)blockIdx.x * E + e] = c;
+  }
 }
 
 // Block-wide exclusive scan of one int per thread (blockDim.x a multiple of
@@ -278,9 +309,10 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
 
 __global__ void __launch_bounds__(1024) scan_and_tiles(const int32_t* __restrict__ hist,
                                                        int n_chunks, int E, int T, int has_shared,
-                                                       int32_t* __restrict__ counts,
+                                                       int TK, int32_t* __restrict__ counts,
                                                        int32_t* __restrict__ offsets,
                                                        int32_t* __restrict__ base,
+                                                       int32_t* __restrict__ perm,
                                                        TileSpec ts, WsHeader* __restrict__ hdr) {
   pdl_wait();
   pdl_trigger();
@@ -314,6 +346,8 @@ __global__ void __launch_bounds__(1024) scan_and_tiles(const int32_t* __restrict
     }
   }
   if (e == E) offsets[E] = total;
+  // rows no copy fills (only when some copy had an expert outside [0, E))
+  for (int r = total + threadIdx.x; r < TK; r += blockDim.x) perm[r] = -1;
   emit_tiles(c, off, E, T, has_shared, ts, sh, hdr);
 }
 
@@ -349,12 +383,9 @@ __global__ void __launch_bounds__(256) chunk_scatter(const int32_t* __restrict__
   __syncthreads();
   const int c0 = blockIdx.x * kChunk;
   const int per_warp = kChunk / kScatterWarps;
-  const int w0 = c0 + warp * per_warp;
+  const int w0 = min(TK, c0 + warp * per_warp);
   const int w1 = min(TK, w0 + per_warp);
-  for (int i = w0 + lane; i < w1; i += 32) {
-    const int e = idx[i];
-    if ((unsigned)e < (unsigned)E) atomicAdd(&cnt[warp][e], 1);
-  }
+  warp_count(idx, w0, w1, E, cnt[warp]);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = base[(size_t)blockIdx.x * E + e];
@@ -376,6 +407,8 @@ __global__ void __launch_bounds__(256) chunk_scatter(const int32_t* __restrict__
       const int row = pre[warp][e] + cnt[warp][e] + rank;
       perm[row] = i;
       inv[i] = row;
+    } else if (live) {
+      inv[i] = -1;   // not placed (expert outside [0, E), reported in the status)
     }
     __syncwarp();
     if (ok && (peers & ((1u << lane) - 1u)) == 0) cnt[warp][e] += __popc(peers);
@@ -407,15 +440,8 @@ __device__ void dispatch_block(const int32_t* __restrict__ idx, int TK, int E, i
   __syncthreads();
   const int per_warp = (TK + nw - 1) / nw;
   const int w0 = min(TK, warp * per_warp), w1 = min(TK, w0 + per_warp);
-  bool bad = false;
-  for (int i = w0 + lane; i < w1; i += 32) {
-    const int e = idx[i];
-    if ((unsigned)e < (unsigned)E)
-      atomicAdd(&cnt[warp * E + e], 1);
-    else
-      bad = true;
-  }
-  if (bad) atomicOr(&hdr->status, kStatusBadIndex);
+  if (warp_count(idx, w0, w1, E, cnt + warp * E) && lane == 0)
+    atomicOr(&hdr->status, kStatusBadIndex);
   __syncthreads();
   const int e = threadIdx.x;   // one thread per expert slot (blockDim > E)
   int c = 0;
@@ -434,6 +460,7 @@ __device__ void dispatch_block(const int32_t* __restrict__ idx, int TK, int E, i
     }
   }
   if (e == E) offsets[E] = total;
+  for (int r = total + threadIdx.x; r < TK; r += blockDim.x) perm[r] = -1;   // unfilled rows
   emit_tiles(c, off, E, T, has_shared, ts, sh, hdr);
   __syncthreads();
   for (int i0 = w0; i0 < w1; i0 += 32) {
@@ -447,6 +474,8 @@ __device__ void dispatch_block(const int32_t* __restrict__ idx, int TK, int E, i
       const int row = pre[warp * E + ei] + cnt[warp * E + ei] + rank;
       perm[row] = i;
       inv[i] = row;
+    } else if (live) {
+      inv[i] = -1;   // not placed (expert outside [0, E), reported in the status)
     }
     __syncwarp();
     if (ok && (peers & ((1u << lane) - 1u)) == 0) cnt[warp * E + ei] += __popc(peers);
@@ -592,13 +621,13 @@ static cudaError_t dispatch_impl(const moe_layer_desc& d, const WsLayout& L, cha
   }
   cudaError_t e = cudaSuccess;
   if (TK > 0)
-    e = launch_pdl(chunk_histogram, dim3(n_chunks), dim3(256), 0, st, idx, TK, d.E, hist,
-                   &hdr->status);
+    e = launch_pdl(chunk_histogram, dim3(n_chunks), dim3(kHistWarps * 32), 0, st, idx, TK, d.E,
+                   hist, &hdr->status);
   else
     e = cudaMemsetAsync(hist, 0, sizeof(int32_t) * (size_t)n_chunks * d.E, st);
   if (e != cudaSuccess) return e;
   e = launch_pdl(scan_and_tiles, dim3(1), dim3(1024), 0, st, (const int32_t*)hist, n_chunks, d.E,
-                 d.T, has_shared, counts, offsets, base, ts, hdr);
+                 d.T, has_shared, TK, counts, offsets, base, perm, ts, hdr);
   if (e != cudaSuccess) return e;
   if (TK > 0)
     e = launch_pdl(chunk_scatter, dim3(n_chunks), dim3(256), 0, st, idx, TK, d.E,
@@ -632,15 +661,15 @@ cudaError_t launch_dispatch_scratch(const moe_layer_desc& d, int n_chunks, int32
   const int TK = d.T * d.K;
   if (TK > 0) {
     count_launch();
-    chunk_histogram<<<n_chunks, 256, 0, st>>>(idx, TK, d.E, hist, &hdr->status);
+    chunk_histogram<<<n_chunks, kHistWarps * 32, 0, st>>>(idx, TK, d.E, hist, &hdr->status);
   } else {
     cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(int32_t) * (size_t)n_chunks * d.E, st);
     if (e != cudaSuccess) return e;
   }
   TileSpec ts{};
   count_launch();
-  scan_and_tiles<<<1, 1024, 0, st>>>(hist, n_chunks, d.E, d.T, d.Ds > 0 ? 1 : 0, counts, offsets,
-                                     base, ts, hdr);
+  scan_and_tiles<<<1, 1024, 0, st>>>(hist, n_chunks, d.E, d.T, d.Ds > 0 ? 1 : 0, TK, counts,
+                                     offsets, base, perm, ts, hdr);
   if (TK > 0) {
     count_launch();
     chunk_scatter<<<n_chunks, 256, 0, st>>>(idx, TK, d.E, base, perm, inv);

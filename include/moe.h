@@ -165,9 +165,10 @@ moe_status moe_topk_from_logits_noisy(const moe_layer_desc* desc, const float* l
  *   topk_idx [T, K] int32 in [0, E) (input);
  *   counts [E], offsets [E + 1], perm [T*K], inv [T*K] int32 outputs:
  *   copy c = t*K + k lands in row inv[c]; perm[row] = c.
- * A copy whose index is outside [0, E) is skipped (counts then sum to less
- * than T*K, and its perm / inv entries are not written); the workspace
- * status word records it, and moe_check_status reports MOE_ERR_INVALID_ARG. */
+ * A copy whose index is outside [0, E) is not placed: counts then sum to
+ * less than T*K, its inv entry is -1 and the rows past the placed copies
+ * hold perm = -1; the workspace status word records it, and moe_check_status
+ * reports MOE_ERR_INVALID_ARG. moe_combine skips copies with inv = -1. */
 moe_status moe_dispatch(const moe_layer_desc* desc, const int32_t* topk_idx, int32_t* counts,
                         int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
                         size_t ws_bytes, moe_stream stream);
@@ -183,10 +184,14 @@ moe_status moe_dispatch(const moe_layer_desc* desc, const int32_t* topk_idx, int
  * process exits. Limit: T*K <= 65536 (plus the usual E <= 512, K <= 16);
  * larger batches return MOE_ERR_UNSUPPORTED without launching. The first
  * call on a device looks up the array's device address (once per device,
- * with that device current): make that first call before any stream
- * capture. All calls share the array, so calls that overlap on the GPU race.
- * Out-of-range indices are skipped (counts then sum to less than T*K) and
- * not reported. Allocates nothing. */
+ * with that device current) and caches it: make that first call before any
+ * stream capture, and do not call it after cudaDeviceReset on that device
+ * (the cached address belongs to the destroyed context). All calls share
+ * the array, so calls that overlap on the GPU race.
+ * Out-of-range indices are handled as in moe_dispatch (inv = -1, perm = -1
+ * past the placed copies, counts summing to less than T*K) but are not
+ * reported through a status word: a caller that cannot trust its indices
+ * checks that counts sum to T*K. Allocates nothing. */
 moe_status moe_dispatch_noalloc(const moe_layer_desc* desc, const int32_t* topk_idx,
                                 int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                                 moe_stream stream);
