@@ -50,9 +50,10 @@ def parse_args():
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default="c2")
     p.add_argument("--T", type=int, default=None)
-    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--no-sweep", action="store_true", help="time the headline workload point only")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--sweep-all", action="store_true", help="also measure every other workload point")
+    p.add_argument("--sweep-only", default=None,
+                   help="comma-separated workload keys the sweep covers (default: all)")
     p.add_argument("--cold-l2", action="store_true",
                    help="sweep points also report the median forward with L2 flushed before each call")
     return p.parse_args()
@@ -316,13 +317,30 @@ def oracle_threads():
         return os.cpu_count() or 1
 
 
-def time_oracle(wl, inp, T, n_tokens, seed):
+def oracle_sample_size(wl, T):
+    """Tokens whose expert FFNs the oracle computes per step: every token up to
+    64, else the seeded sample the workloads name (128 tokens at the prefill
+    scale, 64 otherwise). Routing and dispatch always cover all T tokens."""
+    if T <= 64:
+        return T
+    return 128 if wl.key == "c5" else 64
+
+
+def oracle_step(wl, inp, T, seed):
+    """One step of the CPU baseline: routing and dispatch of all T tokens plus
+    the expert FFNs and combine of a seeded token sample (fp64 oracle).
+    Returns (seconds, tokens computed)."""
     import oracle
-    tokens = mi.sample_tokens(T, n_tokens, seed).numpy()
+    tokens = mi.sample_tokens(T, oracle_sample_size(wl, T), seed).numpy()
     t0 = time.perf_counter()
     oracle.moe_layer_forward(inp["x"], inp["wr"], inp["bias"], inp["w1"], inp["w2"], inp["ws1"],
                              inp["ws2"], wl.K, tokens=tokens)
     return time.perf_counter() - t0, len(tokens)
+
+
+def oracle_sample_text(wl, T, steps):
+    return (f"{steps} steps, each: routing and dispatch of all {T} tokens + expert FFNs and "
+            f"combine of {oracle_sample_size(wl, T)} seeded sample tokens (fp64 numpy oracle)")
 
 
 # ------------------------------------------------------------ reference ---
@@ -333,17 +351,14 @@ def run_reference(args, wl, T):
     host = mi.draw_layer(wl)
     x = mi.draw_x(wl, T)
     inp = widen_all(oracle_inputs(wl, host, x))
-    n = min(T, 16)
     for i in range(args.warmup):
-        time_oracle(wl, inp, T, n, seed=100 + i)
-    times = []
+        oracle_step(wl, inp, T, seed=100 + i)
+    total, done = 0.0, 0
     for i in range(args.steps):
-        dt, n_done = time_oracle(wl, inp, T, n, seed=200 + i)
-        times.append(dt)
-    total = sum(times)
-    value = n * args.steps / total
-    sample = (f"per step: routing of all {T} tokens + expert FFNs of {n} seeded sample tokens "
-              f"(fp64 numpy oracle)")
+        dt, n = oracle_step(wl, inp, T, seed=200 + i)
+        total += dt
+        done += n
+    value = done / total
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -351,7 +366,7 @@ def run_reference(args, wl, T):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(wl, T, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
-                         "sample": sample},
+                         "sample": oracle_sample_text(wl, T, args.steps)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -513,8 +528,61 @@ class Runner:
         nbytes = xh.numel() * xh.element_size()
         return ms, nbytes, yh[0].numel() * yh[0].element_size()
 
+    def timed_gemms(self, steps, warmup=3):
+        """Device time (ms) per pair of the step's two expert-GEMM launches, run
+        again back to back (moe_expert_gemms) on the dispatched rows and tile
+        lists the last forward left in the workspace; CUDA events on the
+        launching stream. None where the layer runs as a single launch."""
+        M = self.M
+        self.step()
+        try:
+            for _ in range(warmup):
+                M.moe_expert_gemms(self.desc, self.weights, self.x, self.ws)
+        except M.MoEError:
+            return None
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(steps):
+            M.moe_expert_gemms(self.desc, self.weights, self.x, self.ws)
+        end.record()
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / steps
+
     def touched(self):
         return int((self.counts > 0).sum().item())
+
+
+def gemm_roofline(R, wl, T, alg, peaks, steps, ms_step):
+    """Roofline of the dominant kernels: the two grouped expert-GEMM launches,
+    timed as a pair in a loop of their own (Runner.timed_gemms). Achieved =
+    the GEMMs' algorithmic FLOPs (tensor-bound) or bytes (HBM-bound) per pair
+    / the measured time per pair. Where the whole layer is one launch, the
+    dominant kernel is that launch and the step time is its time."""
+    gemm_ms = R.timed_gemms(steps)
+    single = gemm_ms is None
+    if single:
+        bound, _ = roofline_bound(alg["flops"], alg["bytes"], peaks)
+        flops, nbytes, t_ms = alg["flops"], alg["bytes"], ms_step
+        kernel = "single-launch decode forward (router, dispatch, expert GEMVs, combine)"
+    else:
+        bound, _ = roofline_bound(alg["gemm_flops"], alg["gemm_bytes"], peaks)
+        flops, nbytes, t_ms = alg["gemm_flops"], alg["gemm_bytes"], gemm_ms
+        kernel = "grouped expert GEMMs (GEMM1 + GeLU, GEMM2; shared expert included)"
+    if bound == "tensor":
+        achieved, peak, unit = flops / (t_ms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = nbytes / (t_ms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    out = {"kernel": kernel, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+           "frac": achieved / peak,
+           # the same against the seconds-long (power-capped) GEMM figure
+           "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                 if bound == "tensor" else None),
+           "ms_per_launch_pair": None if single else gemm_ms,
+           "share_of_step": 1.0 if single else gemm_ms / ms_step,
+           # the kernels' own time cannot exceed the step that contains them
+           "within_step": True if single else gemm_ms <= ms_step * 1.001}
+    return out
 
 
 def run_ours(args, wl, T):
@@ -543,16 +611,7 @@ def run_ours(args, wl, T):
     stages = R.stages(args.steps)
     touched = R.touched()
     alg = algorithmic(wl, T, touched)
-    gemm_ms = stages["gemm1"] + stages["gemm2"]
-    bound, _ = roofline_bound(alg["gemm_flops"], alg["gemm_bytes"], peaks)
-    if bound == "tensor":
-        achieved = alg["gemm_flops"] / (gemm_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops"]
-        unit = "TFLOP/s"
-    else:
-        achieved = alg["gemm_bytes"] / (gemm_ms / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        unit = "GB/s"
+    rl = gemm_roofline(R, wl, T, alg, peaks, args.steps, ms_step)
     lbound, t_roof = roofline_bound(alg["flops"], alg["bytes"], peaks)
 
     e2e_ms, h2d, d2h = R.e2e(args.steps, args.warmup, world, device)
@@ -564,15 +623,9 @@ def run_ours(args, wl, T):
         "data": "synthetic (seeded: x ~ N(0,1), weights ~ N(0,1/fan_in) in bf16, Zipf logit skew "
                 "as a bias input where the workload has one)",
         "config": workload_config(wl, T, world),
-        "roofline": {"kernel": "grouped expert GEMMs (GEMM1 + GeLU, GEMM2; shared expert included)",
-                     "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak,
-                     # the same against the seconds-long (power-capped) GEMM figure
-                     "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
-                                           if bound == "tensor" else None),
-                     "traffic": measured_traffic(wl, T),
-                     "traffic_unit": "DRAM bytes per launch (mean of GEMM1 and GEMM2)", "peak_source": peaks_src,
-                     "ms_per_launch_pair": gemm_ms},
+        "roofline": dict(rl, traffic=measured_traffic(wl, T),
+                         traffic_unit="DRAM bytes per launch (mean of GEMM1 and GEMM2)",
+                         peak_source=peaks_src),
         "layer_roofline": {"bound": lbound, "t_roof_ms": 1e3 * t_roof, "frac": 1e3 * t_roof / ms_step,
                            "flops": alg["flops"], "bytes": alg["bytes"], "experts_touched": touched},
         "stages_ms": stages,
@@ -582,7 +635,8 @@ def run_ours(args, wl, T):
         "clocks": clocks,
     }
     if not args.no_sweep and world == 1:
-        line["sweep"] = sweep(M, wl, dev, T, peaks, args.sweep_all, args.cold_l2)
+        only = args.sweep_only.split(",") if args.sweep_only else None
+        line["sweep"] = sweep(M, wl, dev, T, peaks, only, args.cold_l2)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, host, R.x_host, T)
     if rank == 0:
@@ -600,10 +654,17 @@ def measure_point(M, wl, dev, T, peaks, steps=20, warmup=5, cold=False):
     bound, t_roof = roofline_bound(alg["flops"], alg["bytes"], peaks)
     ms_step = ms / steps
     graph_ms = R.timed_graph(steps, warmup) / steps
+    rl = gemm_roofline(R, wl, T, alg, peaks, steps, ms_step)
     out = {"workload": wl.key, "T": T, "tokens_per_s": T / (ms_step / 1e3), "us_per_step": 1e3 * ms_step,
            "graph_us_per_step": 1e3 * graph_ms, "graph_frac": 1e3 * t_roof / graph_ms,
            "bound": bound, "roofline_us": 1e6 * t_roof, "frac": 1e3 * t_roof / ms_step,
-           "experts_touched": R.touched(), "stages_us": {k: 1e3 * v for k, v in st.items()}}
+           "experts_touched": R.touched(),
+           "dominant": {"kernel": rl["kernel"], "bound": rl["bound"], "achieved": rl["achieved"],
+                        "unit": rl["unit"], "frac": rl["frac"],
+                        "us_per_launch_pair": (None if rl["ms_per_launch_pair"] is None
+                                               else 1e3 * rl["ms_per_launch_pair"]),
+                        "within_step": rl["within_step"]},
+           "stages_us": {k: 1e3 * v for k, v in st.items()}}
     if cold:
         cold_ms = R.timed_cold(max(steps, 50))
         out["cold_l2_us_per_step"] = 1e3 * cold_ms
@@ -611,33 +672,42 @@ def measure_point(M, wl, dev, T, peaks, steps=20, warmup=5, cold=False):
     return out
 
 
-def sweep(M, wl, dev, T_main, peaks, all_workloads, cold=False):
-    out = [measure_point(M, wl, dev, T, peaks, cold=cold) for T in wl.Ts if T != T_main]
-    if all_workloads:
-        for key in ("c3", "c4", "c5", "c1"):
-            if key == wl.key:
-                continue
-            w2 = mi.WORKLOADS[key]
+def sweep(M, wl, dev, T_main, peaks, only=None, cold=False):
+    """Every point of every workload (the headline point excepted), each
+    workload's weights resident only while its points run."""
+    keys = ["c1", "c2", "c3", "c4", "c5"] if not only else only
+    out = []
+    for key in keys:
+        w2 = mi.WORKLOADS[key]
+        if key == wl.key:
+            d2 = dev
+        else:
             host = mi.draw_layer(w2)
             d2 = {k: (v.cuda() if v is not None else None) for k, v in host.items()}
-            for T in w2.Ts:
-                out.append(measure_point(M, w2, d2, T, peaks, cold=cold))
+            del host
+        for T in w2.Ts:
+            if key == wl.key and T == T_main:
+                continue
+            out.append(measure_point(M, w2, d2, T, peaks, cold=cold))
+        if key != wl.key:
             del d2
             torch.cuda.empty_cache()
     return out
 
 
-def cpu_baseline(wl, host, x, T, target_s=15.0):
-    """The oracle on the host cores: a short calibration run, then a sample
-    sized to about target_s seconds (the whole batch if that is less)."""
+def cpu_baseline(wl, host, x, T, target_s=12.0):
+    """The oracle on the host cores, with the reference arm's per-step program
+    (oracle_step), repeated until about target_s seconds of CPU work."""
     inp = widen_all(oracle_inputs(wl, host, x))
-    n0 = min(T, 64)
-    dt0, _ = time_oracle(wl, inp, T, n0, seed=6)
-    n = T if dt0 * T / n0 <= 2 * target_s else max(n0, int(n0 * target_s / max(dt0, 1e-3)))
-    dt, n_done = time_oracle(wl, inp, T, n, seed=7)
-    return {"value": n_done / dt, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"routing of all {T} tokens + expert FFNs of {n_done} seeded sample tokens "
-                      f"(fp64 numpy oracle, {dt:.1f} s)"}
+    oracle_step(wl, inp, T, seed=99)          # warm-up (first touch of the weights)
+    total, done, steps = 0.0, 0, 0
+    while steps < 1 or total < target_s:
+        dt, n = oracle_step(wl, inp, T, seed=300 + steps)
+        total += dt
+        done += n
+        steps += 1
+    return {"value": done / total, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": oracle_sample_text(wl, T, steps) + f", {total:.1f} s"}
 
 
 def main():

@@ -26,6 +26,7 @@ EXPORTED = (
     "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
     "moe_expert_stats", "moe_bias_update",
     "moe_check_status", "moe_status_string", "moe_kernel_launch_count", "moe_dispatch_noalloc",
+    "moe_expert_gemms",
 )
 
 
@@ -86,6 +87,7 @@ def _load() -> ctypes.CDLL:
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_kernel_launch_count": (ctypes.c_uint64, []),
         "moe_dispatch_noalloc": (ctypes.c_int, [D, P, P, P, P, P, P]),
+        "moe_expert_gemms": (ctypes.c_int, [D, ctypes.POINTER(MoELayerWeights), P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -230,6 +232,13 @@ def moe_layer_forward_profiled(desc, weights: MoELayerWeights, x, y, routing: Op
                                           _p(ws), ws.numel() if ws is not None else 0,
                                           _stream(stream), arr, len(events)),
            "moe_layer_forward_profiled")
+
+
+def moe_expert_gemms(desc, weights: MoELayerWeights, x, ws, stream=None) -> None:
+    """The expert-GEMM launches of the last moe_layer_forward on `ws` again (timing)."""
+    _check(lib.moe_expert_gemms(ctypes.byref(desc), ctypes.byref(weights), _p(x), _p(ws),
+                                ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_expert_gemms")
 
 
 def moe_expert_stats(desc, counts, straggler_mask, ws, stream=None) -> dict:

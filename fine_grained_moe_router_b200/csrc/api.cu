@@ -582,6 +582,34 @@ static moe_status layer_forward_impl(const moe_layer_desc* desc, const moe_layer
   auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
 
   const bool tc = d.dtype == MOE_BF16;
+  // A handful of bf16 tokens: the whole layer in one cooperative launch
+  // (router, selection, dispatch, both expert layers, combine).
+  if (tc && decode_eligible(d)) {
+    DecodeBuffers b{};
+    b.x = x;
+    b.w_router = W.w_router;
+    b.w1 = W.w1;
+    b.w2 = W.w2;
+    b.ws1 = W.ws1;
+    b.ws2 = W.ws2;
+    b.bias = W.expert_bias;
+    b.noise = noise;
+    b.y = y;
+    b.logits = R.logits ? R.logits : reinterpret_cast<float*>(w + L.logits);
+    b.idx = idx;
+    b.tw = tw;
+    b.counts = counts;
+    b.offsets = offsets;
+    b.perm = perm;
+    b.inv = inv;
+    b.hm = w + L.hm;
+    b.hs = w + L.hs;
+    b.hdr = reinterpret_cast<WsHeader*>(w + L.hdr);
+    MOE_CUDA_TRY(mark(0));
+    MOE_CUDA_TRY(launch_decode_forward(d, b, st));
+    for (int i = 1; i < kForwardEvents; ++i) MOE_CUDA_TRY(mark(i));
+    return MOE_OK;
+  }
   // bf16 decode batches with a shared expert: its GEMMs go to the side stream
   // first. Measured on B200: 2-6% faster from T = 16 on; slower at T = 1
   // (the fork and join cost more than the overlap gains) and on CTA-pair
@@ -662,6 +690,28 @@ moe_status moe_layer_forward_profiled(const moe_layer_desc* desc,
   return layer_forward_impl(desc, weights, x, y, routing_or_null, ws, ws_bytes,
                             static_cast<cudaStream_t>(stream),
                             reinterpret_cast<cudaEvent_t const*>(stage_events), n_events);
+}
+
+moe_status moe_expert_gemms(const moe_layer_desc* desc, const moe_layer_weights* weights,
+                            const void* x, void* ws, size_t ws_bytes, moe_stream stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc& d = *desc;
+  MOE_TRY(check_ws(d, ws, ws_bytes));
+  if (!weights) return MOE_ERR_INVALID_ARG;
+  if (d.T == 0) return MOE_OK;
+  if (d.dtype != MOE_BF16 || decode_eligible(d)) return MOE_ERR_UNSUPPORTED;
+  const moe_layer_weights& W = *weights;
+  MOE_TRY(check_ptrs({x, W.w1, W.w2}));
+  if (d.Ds > 0) MOE_TRY(check_ptrs({W.ws1, W.ws2}));
+  const WsLayout L = workspace_layout(d);
+  char* w = static_cast<char*>(ws);
+  // the same choice as moe_layer_forward: a shared expert on the side stream
+  // is not part of the caller-stream launches
+  const bool side = d.Ds > 0 && !L.sp.pair && d.T >= kSideStreamMinT;
+  void* ys = d.Ds > 0 ? static_cast<void*>(w + L.ys) : nullptr;
+  return run_grouped_ffn(d, L, w, x, reinterpret_cast<const int32_t*>(w + L.perm), W.w1, W.w2,
+                         W.ws1, W.ws2, w + L.yr, ys, static_cast<cudaStream_t>(stream),
+                         /*split=*/true, nullptr, /*with_shared=*/!side);
 }
 
 moe_status moe_expert_stats(const moe_layer_desc* desc, const int32_t* counts,

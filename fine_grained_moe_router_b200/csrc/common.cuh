@@ -14,6 +14,7 @@ namespace moe {
 constexpr int kMaxK = 16;
 constexpr int kMaxE = 512;
 constexpr int kForwardEvents = 6;   // stage events of moe_layer_forward_profiled
+constexpr int kDecodeMaxT = 4;      // tokens of the single-launch decode forward (at most)
 
 // Status bits written by kernels into the workspace header.
 constexpr uint32_t kStatusTimeout = 1u;

@@ -338,7 +338,8 @@ __device__ __forceinline__ void epilogue_bar_sync() {   // the kEpiWarps epilogu
 // splits in split order, applies the GeLU and stores the bf16 output. Thread
 // = output column `col`; the two warps of a lane quarter take alternate rows.
 // Arrivals are counted in the split-0 tile of the list (one counter per CTA
-// of a pair), which the dispatch step writes as 0 every forward. All
+// of a pair), which the dispatch step writes as 0 every forward and the last
+// arrival puts back to 0. All
 // epilogue warps call this together (it holds named barriers).
 constexpr int kFixRows = 4;   // rows per thread and round of loads
 
@@ -349,7 +350,11 @@ __device__ __noinline__ void split_fixup(const Args& args, const Tile& tl, const
   epilogue_bar_sync();
   if (threadIdx.x == 0) {
     int* arrivals = const_cast<int*>(&args.tiles[tl.first_split].arrivals[rank]);
-    *owner = (atomicAdd(arrivals, 1) == S.splits - 1) ? 1 : 0;
+    const bool last = atomicAdd(arrivals, 1) == S.splits - 1;
+    // every split has arrived, so nothing else touches the counter in this
+    // launch: leave it at zero for the next launch on the same tile list
+    if (last) *arrivals = 0;
+    *owner = last ? 1 : 0;
   }
   epilogue_bar_sync();
   if (!*owner) return;

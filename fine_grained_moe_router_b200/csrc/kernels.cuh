@@ -88,6 +88,25 @@ cudaError_t launch_grouped_gemm_simt(int dtype, bool gelu, const SimtProblem& ro
 cudaError_t launch_combine(const moe_layer_desc& d, const void* y_rows, const float* w,
                            const int32_t* inv, const void* y_shared, void* y, cudaStream_t st,
                            int rows_parts = 1, int shared_parts = 1);
+// Buffers of the single-launch decode forward (bf16 layers, T <= kDecodeMaxT):
+// inputs, the output y, the routing outputs (caller's or workspace buffers),
+// the first layer's outputs Hm [T*K, D] and Hs [T, Ds] in the workspace, and
+// the workspace header (status word, grid barrier counters).
+struct DecodeBuffers {
+  const void *x, *w_router, *w1, *w2, *ws1, *ws2;
+  const float* bias;    // nullable
+  const float* noise;   // nullable
+  void* y;
+  float* logits;
+  int32_t *idx, *counts, *offsets, *perm, *inv;
+  float* tw;
+  void *hm, *hs;
+  WsHeader* hdr;
+};
+// True when the shape runs as one cooperative launch on this device.
+bool decode_eligible(const moe_layer_desc& d);
+cudaError_t launch_decode_forward(const moe_layer_desc& d, const DecodeBuffers& b,
+                                  cudaStream_t st);
 cudaError_t launch_bias_update(const moe_layer_desc& d, const int32_t* counts, float* bias,
                                float gamma, cudaStream_t st);
 cudaError_t launch_expert_stats(const moe_layer_desc& d, const int32_t* counts, uint8_t* mask,

@@ -252,6 +252,17 @@ moe_status moe_layer_forward_profiled(const moe_layer_desc* desc,
                                       size_t ws_bytes, moe_stream stream,
                                       void* const* stage_events, int n_events);
 
+/* The two grouped expert-GEMM launches (first layer with its GeLU, second
+ * layer) of the most recent moe_layer_forward on this workspace, run again
+ * on the dispatched rows and tile lists that forward left in it, for timing
+ * the dominant kernels of a step in isolation. Same desc, weights and x as
+ * that forward; overwrites only the workspace's expert outputs. bf16 layers
+ * that take the multi-launch path only (MOE_ERR_UNSUPPORTED otherwise); a
+ * shared expert that ran on the library's side stream is not included.
+ * "MoE architecture in production" §3.1 (experts of Linear, GeLU, Linear). */
+moe_status moe_expert_gemms(const moe_layer_desc* desc, const moe_layer_weights* weights,
+                            const void* x, void* ws, size_t ws_bytes, moe_stream stream);
+
 /* Load statistics from counts [E] (device). "Kimi K3 专家路由不均衡诊断" §三
  * (analyze_batch_routing, compute_gini_coefficient); overflow copies are
  * counted, never dropped (§五). straggler_mask_or_null [E] uint8 device

@@ -69,3 +69,42 @@ def test_roofline_bound_picks_the_slower_resource():
 def _fb(bench, w, T, touched):
     a = bench.algorithmic(w, T, touched)
     return {"flops": a["flops"], "nbytes": a["bytes"], "peaks": PEAKS}
+
+
+class _FakeRunner:
+    def __init__(self, gemm_ms):
+        self.gemm_ms = gemm_ms
+
+    def timed_gemms(self, steps):
+        return self.gemm_ms
+
+
+def test_dominant_kernel_roofline_from_the_gemm_loop():
+    """achieved = the GEMMs' algorithmic FLOPs / their own loop time; the pair
+    must fit in the step that contains it, and a single-launch step is its
+    own dominant kernel."""
+    import bench
+    wl = bench.mi.WORKLOADS["c2"]
+    a = bench.algorithmic(wl, 4096, 8)
+    peaks = dict(PEAKS, bf16_tflops_sustained=1425.2)
+    r = bench.gemm_roofline(_FakeRunner(1.60), wl, 4096, a, peaks, 20, ms_step=1.75)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(a["gemm_flops"] / 1.60e-3 / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / 1656.9)
+    assert r["within_step"] and r["share_of_step"] == pytest.approx(1.60 / 1.75)
+    assert not bench.gemm_roofline(_FakeRunner(1.80), wl, 4096, a, peaks, 20, 1.75)["within_step"]
+    d = bench.algorithmic(bench.mi.WORKLOADS["c3"], 1, 8)
+    r = bench.gemm_roofline(_FakeRunner(None), bench.mi.WORKLOADS["c3"], 1, d, peaks, 20, 0.040)
+    assert r["bound"] == "hbm" and r["achieved"] == pytest.approx(d["bytes"] / 40e-6 / 1e9)
+    assert r["share_of_step"] == 1.0 and r["ms_per_launch_pair"] is None
+
+
+def test_reference_arm_and_cpu_baseline_share_one_sampling_rule():
+    import bench
+    wl = bench.mi.WORKLOADS
+    assert bench.oracle_sample_size(wl["c2"], 8) == 8
+    assert bench.oracle_sample_size(wl["c2"], 4096) == 64
+    assert bench.oracle_sample_size(wl["c5"], 16384) == 128
+    # both arms describe the same per-step program
+    t = bench.oracle_sample_text(wl["c2"], 4096, 20)
+    assert "all 4096 tokens" in t and "64 seeded sample tokens" in t
