@@ -26,7 +26,7 @@ EXPORTED = (
     "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
     "moe_expert_stats", "moe_bias_update",
     "moe_check_status", "moe_status_string", "moe_kernel_launch_count", "moe_dispatch_noalloc",
-    "moe_expert_gemms",
+    "moe_expert_gemms", "moe_gather_rows", "moe_ep_local_order",
 )
 
 
@@ -88,6 +88,10 @@ def _load() -> ctypes.CDLL:
         "moe_kernel_launch_count": (ctypes.c_uint64, []),
         "moe_dispatch_noalloc": (ctypes.c_int, [D, P, P, P, P, P, P]),
         "moe_expert_gemms": (ctypes.c_int, [D, ctypes.POINTER(MoELayerWeights), P, P, S, P]),
+        "moe_gather_rows": (ctypes.c_int, [P, ctypes.c_int64, P, ctypes.c_int32, ctypes.c_int64,
+                                           ctypes.c_int64, P, P]),
+        "moe_ep_local_order": (ctypes.c_int, [P, ctypes.c_int32, ctypes.c_int32, P, P, P,
+                                              ctypes.c_int64, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -239,6 +243,22 @@ def moe_expert_gemms(desc, weights: MoELayerWeights, x, ws, stream=None) -> None
     _check(lib.moe_expert_gemms(ctypes.byref(desc), ctypes.byref(weights), _p(x), _p(ws),
                                 ws.numel() if ws is not None else 0, _stream(stream)),
            "moe_expert_gemms")
+
+
+def moe_gather_rows(src, idx, divisor: int, dst, stream=None) -> None:
+    """dst[r] = src[idx[r] // divisor] for every row of dst (row-major 2-D tensors)."""
+    row_bytes = dst[0].numel() * dst.element_size() if dst.shape[0] else 16
+    _check(lib.moe_gather_rows(_p(src), src.shape[0], _p(idx), int(divisor), dst.shape[0],
+                               row_bytes, _p(dst), _stream(stream)), "moe_gather_rows")
+
+
+def moe_ep_local_order(recv_counts, offsets, perm, inv, stream=None) -> None:
+    """Expert-major order of the rows received from G ranks (recv_counts [G, El] int32)."""
+    G, El = recv_counts.shape
+    _check(lib.moe_ep_local_order(_p(recv_counts), G, El, _p(offsets),
+                                  _p(perm) if perm.numel() else None,
+                                  _p(inv) if inv.numel() else None, perm.numel(),
+                                  _stream(stream)), "moe_ep_local_order")
 
 
 def moe_expert_stats(desc, counts, straggler_mask, ws, stream=None) -> dict:

@@ -563,6 +563,20 @@ __global__ void __launch_bounds__(256) gather_rows(const uint4* __restrict__ x,
     gather_row(x, perm, TK, K, row_vecs, xp, row, threadIdx.x & 31);
 }
 
+// The same copy for any rows: dst[r] = src[idx[r] / divisor] for r < n_rows,
+// idx values checked against idx_bound (rows with an index outside it are
+// left unwritten).
+__global__ void __launch_bounds__(256) gather_rows_any(const uint4* __restrict__ src,
+                                                       const int32_t* __restrict__ idx,
+                                                       int idx_bound, int n_rows, int divisor,
+                                                       int row_vecs, uint4* __restrict__ dst) {
+  pdl_wait();
+  pdl_trigger();
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < n_rows; row += warps)
+    gather_row(src, idx, idx_bound, divisor, row_vecs, dst, row, threadIdx.x & 31);
+}
+
 static TileSpec make_tile_spec(const moe_layer_desc& d, const WsLayout& L, char* ws,
                                bool tc_tiles, bool split) {
   TileSpec ts;
@@ -682,6 +696,17 @@ cudaError_t launch_tiles_from_offsets(const moe_layer_desc& d, const WsLayout& L
   const TileSpec ts = make_tile_spec(d, L, ws, tc_tiles, /*split=*/false);
   return launch_pdl(tiles_from_offsets, dim3(1), dim3(1024), 0, st, offsets, d.E, d.T,
                     d.Ds > 0 ? 1 : 0, ts, reinterpret_cast<WsHeader*>(ws + L.hdr));
+}
+
+cudaError_t launch_gather_rows_raw(const void* src, int idx_bound, const int32_t* idx, int n_rows,
+                                   int divisor, int row_vecs, void* dst, cudaStream_t st) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int blocks = (int)std::min<long long>(((long long)n_rows + 7) / 8, (long long)sms * 8);
+  return launch_pdl(gather_rows_any, dim3(std::max(1, blocks)), dim3(256), 0, st,
+                    static_cast<const uint4*>(src), idx, idx_bound, n_rows, divisor, row_vecs,
+                    static_cast<uint4*>(dst));
 }
 
 cudaError_t launch_gather_rows(const moe_layer_desc& d, const void* x, const int32_t* perm,

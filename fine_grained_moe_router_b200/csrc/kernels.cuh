@@ -79,6 +79,13 @@ cudaError_t launch_tiles_from_offsets(const moe_layer_desc& d, const WsLayout& L
                                       const int32_t* offsets, bool tc_tiles, cudaStream_t st);
 cudaError_t launch_gather_rows(const moe_layer_desc& d, const void* x, const int32_t* perm,
                                void* xp, int num_sms, cudaStream_t st);
+// dst[r] = src[idx[r] / divisor] (row_vecs 16-byte vectors a row) for r < n_rows; idx
+// values at or above idx_bound (or negative) leave the row unwritten.
+cudaError_t launch_gather_rows_raw(const void* src, int idx_bound, const int32_t* idx, int n_rows,
+                                   int divisor, int row_vecs, void* dst, cudaStream_t st);
+// Expert-major order of the rows one rank receives (see ep.cu).
+cudaError_t launch_ep_local_order(const int32_t* cnt, int G, int El, int32_t* offsets,
+                                  int32_t* perm, int32_t* inv, int capacity, cudaStream_t st);
 cudaError_t launch_grouped_gemm_simt(int dtype, bool gelu, const SimtProblem& routed,
                                      const SimtProblem& shared, int E, const Tile* tiles,
                                      const int* n_tiles, int max_tiles, int max_n,

@@ -285,6 +285,35 @@ moe_status moe_expert_stats(const moe_layer_desc* desc, const int32_t* counts,
 moe_status moe_bias_update(const moe_layer_desc* desc, const int32_t* counts, float* bias,
                            float gamma, moe_stream stream);
 
+/* Expert parallelism ("Kimi K3 fine-grained MoE ...", section "物理通信拓扑":
+ * dispatch All-to-All, local experts, combine All-to-All; "MoE architecture
+ * in production" §3.2). Ranks own contiguous ranges of experts; the
+ * exchanges themselves are the caller's collective (NCCL All-to-All into
+ * each rank's own buffers); these two calls prepare the rows around them.
+ *
+ * Row gather: dst[r] = src[idx[r] / divisor] for r < n_rows, rows of
+ * row_bytes bytes (a multiple of 16; src, dst 16-byte aligned). idx values
+ * outside [0, src_rows * divisor) leave their row unwritten. With the
+ * dispatch's perm and divisor K it fills an All-to-All send buffer from x;
+ * with moe_ep_local_order's inv and divisor 1 it puts expert outputs back
+ * in receive order. */
+moe_status moe_gather_rows(const void* src, int64_t src_rows, const int32_t* idx,
+                           int32_t divisor, int64_t n_rows, int64_t row_bytes, void* dst,
+                           moe_stream stream);
+
+/* Order of the rows a rank receives from G source ranks for its El
+ * experts: recv_counts [G, El] int32 (device; rows of expert e from source
+ * s), the rows arriving source by source, each source's in ascending expert
+ * order. Outputs (device): offsets [El + 1], the expert-major segment of
+ * each local expert (expert e's rows of source 0, then source 1, ...);
+ * perm [R] (expert-major position -> receive position) and inv [R] (the
+ * inverse), R = sum(recv_counts) <= rows_capacity (entries past the
+ * capacity are not written; perm / inv may be NULL when rows_capacity = 0).
+ * Limits: G, El <= 1024, G * El <= 4096. */
+moe_status moe_ep_local_order(const int32_t* recv_counts, int32_t G, int32_t El,
+                              int32_t* offsets, int32_t* perm, int32_t* inv,
+                              int64_t rows_capacity, moe_stream stream);
+
 /* Reads and clears the workspace status word (synchronises `stream`):
  * MOE_OK; MOE_ERR_TIMEOUT if a bounded device wait ran out (this takes
  * precedence); MOE_ERR_INVALID_ARG if a dispatch met a top-K index outside
