@@ -26,15 +26,17 @@
 //            Yr[inv[t,k], h] + S[t, h] ("Kimi K3 ...", section "物理通信拓扑",
 //            combine phase) follows in the same CTA, k ascending, fp32.
 //
-// Weight streaming: a warp takes whole weight rows (rows dealt round-robin
-// over the CTA's 16 warps) and streams them straight from HBM into
-// registers with 16-byte non-caching loads, in segments of a few vectors per
-// lane, double-buffered: the next segment's loads are in flight while the
-// current one is multiplied (fused bf16 x bf16 + fp32 multiply-adds) with
-// the activation rows, which are staged once per phase in shared memory (x,
-// then the first layer's outputs). The lanes' partial sums of a row are added
-// by a shuffle butterfly. Every order of additions is fixed, so results are
-// deterministic. The only CTA-wide synchronisation is at phase boundaries.
+// Weight streaming: a phase's weight rows are cut into chunks of 32 16-byte
+// vectors, and each warp of the CTA takes an equal contiguous range of them
+// (whatever the rows' lengths), copied from HBM with cp.async into a private
+// ring of shared-memory stages of 4 KB, a few segments in flight while one
+// is multiplied (fused bf16 x bf16 + fp32 multiply-adds) with the activation
+// rows, which are staged once per phase in shared memory (x, then the first
+// layer's outputs). The lanes' partial sums of a row are added by a shuffle
+// butterfly; a row that a warp boundary cuts is finished after the phase
+// from the warps' sums, in warp order. Every order of additions is fixed, so
+// results are deterministic. The only CTA-wide synchronisation is at phase
+// boundaries.
 //
 // Every wait is bounded in time (the grid barriers): on expiry the CTA sets
 // kStatusTimeout in the workspace and skips the rest of the layer. The grid
@@ -167,38 +169,60 @@ __device__ __forceinline__ void grid_arrive(const Params& p) {
 enum Out : int { kLogits = 0, kHs, kHm, kYr, kS };
 
 // One matrix's rows [r0, r1) for this CTA (row length L): a job. A phase is a
-// list of jobs whose rows are dealt round-robin over a set of warps (job by
-// job), each against A <= kDecodeMaxT activation rows staged in shared
-// memory (16-byte vector offsets act[0..A) from the staging base). Row r's
-// result for activation row a goes to the output `out`: logits[a, r]; Hs[a,
-// r] or Hm[seg_off + a, r] after the GeLU (bf16); Yr (ycache[r - h0, seg_off
-// + a]) or S (scache[r - h0, a]).
+// list of jobs, each against A <= kDecodeMaxT activation rows staged in
+// shared memory (16-byte vector offsets act[0..A) from the staging base). Row
+// r's result for activation row a goes to the output `out`: logits[a, r];
+// Hs[a, r] or Hm[seg_off + a, r] after the GeLU (bf16); Yr (ycache[r - h0,
+// seg_off + a]) or S (scache[r - h0, a]).
+//
+// The phase's weight bytes are cut into chunks of 32 16-byte vectors (one
+// per lane; a row of nvec vectors takes cpr = ceil(nvec / 32) chunks, the
+// last one masked past nvec), numbered job by job, row by row; chunk c0 is
+// the job's first. Warp wi of nw takes the contiguous chunks [C wi / nw,
+// C (wi + 1) / nw) of the phase's C, so every warp streams the same number of
+// bytes whatever the rows' lengths; a row cut by a warp boundary is finished
+// after the phase from the warps' partial sums, added in warp order.
 struct RowJob {
   const __nv_bfloat16* w;
   int r0, r1, L;
   int act[kDecodeMaxT];
   int A, out, seg_off, h0;
+  int nvec, cpr, c0;
+};
+
+// Fills nvec, cpr and c0 of a phase's jobs; returns the phase's chunks.
+__device__ __forceinline__ int number_chunks(RowJob* jobs, int n) {
+  int c = 0;
+  for (int j = 0; j < n; ++j) {
+    jobs[j].nvec = jobs[j].L / 8;
+    jobs[j].cpr = (jobs[j].nvec + 31) / 32;
+    jobs[j].c0 = c;
+    c += (jobs[j].r1 - jobs[j].r0) * jobs[j].cpr;
+  }
+  return c;
+}
+
+// A row that a warp boundary cuts: each warp's sum over its part (slot 0:
+// the first row of the warp's range, slot 1: the last). `head`: the part
+// holds the row's first chunk; `tail`: its last.
+struct Partial {
+  int valid, head, tail, job, row;
+  float v[kDecodeMaxT];
 };
 
 constexpr int kMaxJobs = kMaxCopies + 1;   // every touched expert + the shared expert
-constexpr int kVpl = 8;                    // 16-byte vectors per lane per stage (4 KB a warp)
+// A CTA's share of the first layer's rows (ns * D rows of ns <= 64 touched
+// experts, over at least 64 CTAs) is at most D rows, so it meets at most two
+// experts' row blocks.
+constexpr int kMaxG1Jobs = 4;
+constexpr int kMinCtas = kMaxCopies;
+constexpr int kVpl = 8;                    // chunks per lane per stage (4 KB a warp)
 // shared memory of the per-warp rings with kStages stages
 constexpr size_t ring_bytes(int stages) { return (size_t)kWarps * stages * kVpl * 32 * 16; }
 
-template <int kA>
-__device__ __forceinline__ void row_out(const RowJob& jb, const Params& p, int r, float (&sum)[kA],
-                                        float* ycache, float* scache) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-    for (int a = 0; a < kA; ++a) sum[a] += __shfl_xor_sync(0xffffffffu, sum[a], o);
-  if (lane >= jb.A) return;
-  float v = sum[0];
-#pragma unroll
-  for (int a = 1; a < kA; ++a)
-    if (lane == a) v = sum[a];
-  const int a = lane;
+// Result v of row r (of job jb) for activation row a.
+__device__ __forceinline__ void emit(const RowJob& jb, const Params& p, int r, int a, float v,
+                                     float* ycache, float* scache) {
   switch (jb.out) {
     case kLogits:
       p.logits[(size_t)a * p.E + r] = v;
@@ -225,75 +249,87 @@ __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-// Position in a warp's stream of segments over a job list: job j, segment k
-// of the job; a segment is up to 32 * kVpl vectors of one row, lane l taking
-// vectors l, l + 32, ... of it.
+// Position in a warp's chunk range: job j, row `row` of the job, chunk cc of
+// the row, `left` chunks to go.
 struct Cursor {
-  int j, k;
+  int j, row, cc, left;
 };
 
-// Rows of job jb that warp wi of nw takes, and segments per row.
-__device__ __forceinline__ int job_rows(const RowJob& jb, int wi, int nw) {
-  const int n = jb.r1 - jb.r0;
-  return n > wi ? (n - wi + nw - 1) / nw : 0;
-}
-__device__ __forceinline__ int job_spr(const RowJob& jb) {
-  return (jb.L / 8 + 32 * kVpl - 1) / (32 * kVpl);
-}
-// Moves c to the next segment (k + 1, or the first segment of the next job
-// with rows for this warp); c.j == n_jobs at the end.
-__device__ __forceinline__ void advance(Cursor& c, const RowJob* jobs, int n_jobs, int wi, int nw) {
-  ++c.k;
-  while (c.j < n_jobs && c.k >= job_rows(jobs[c.j], wi, nw) * job_spr(jobs[c.j])) {
-    ++c.j;
-    c.k = 0;
-  }
+// Cursor at chunk c of the phase with `left` chunks to go.
+__device__ __forceinline__ Cursor seek(const RowJob* jobs, int n_jobs, int c, int left) {
+  Cursor k{0, 0, 0, left};
+  if (left <= 0) return k;
+  // the last job starting at or before c (jobs without rows share their c0
+  // with the next one)
+  while (k.j + 1 < n_jobs && jobs[k.j + 1].c0 <= c) ++k.j;
+  const int local = c - jobs[k.j].c0;
+  k.row = local / jobs[k.j].cpr;
+  k.cc = local % jobs[k.j].cpr;
+  return k;
 }
 
-// The calling warp's share (warp wi of nw) of a phase's job list, as a
-// stream of segments: each lane copies its own vectors of the next segments
-// into the warp's private ring of kStages stages with cp.async (kStages - 1
-// segments in flight while one is multiplied; a lane reads back only what it
-// copied itself, so no synchronisation is needed), and the stream runs on
-// across job boundaries. prime() puts the first kStages - 1 segments in
-// flight (weights only: it may run before the activations are staged);
-// run() multiplies the whole stream. Each row keeps two partial sums per
-// activation row (even and odd vectors), added before the butterfly.
+// Moves k past `run` chunks of its current row (run <= the chunks left in
+// the row); at the row's end to the next row, or the next job with rows.
+__device__ __forceinline__ void step(Cursor& k, const RowJob* jobs, int n_jobs, int run, int cpr,
+                                     int rows) {
+  k.left -= run;
+  k.cc += run;
+  if (k.cc < cpr) return;
+  k.cc = 0;
+  if (++k.row < rows) return;
+  k.row = 0;
+  do ++k.j;
+  while (k.j < n_jobs && jobs[k.j].r1 == jobs[k.j].r0);
+}
+
+// The calling warp's range of a phase's chunks as a stream: each lane copies
+// its own vectors of the next segments (kVpl chunks) into the warp's private
+// ring of kStages stages with cp.async (kStages - 1 segments in flight while
+// one is multiplied; a lane reads back only what it copied itself, so no
+// synchronisation is needed). prime() puts the first kStages - 1 segments in
+// flight (weights only: it may run before the activations are staged); run()
+// multiplies the whole range. A segment is walked in runs of chunks of one
+// row; each row keeps two partial sums per activation row (alternate chunks
+// of a run), added before the lanes' butterfly.
 template <int kStages>
 struct JobStream {
   const RowJob* jobs;
-  int n_jobs, wi, nw, n;
+  int n_jobs, wi, n;
   Cursor in, out;
   uint4* my_ring;
   uint32_t my_ring_s;
 
-  __device__ void init(const RowJob* jobs_, int n_jobs_, int wi_, int nw_, uint4* ring) {
+  __device__ void init(const RowJob* jobs_, int n_jobs_, int chunks, int wi_, int nw,
+                       uint4* ring) {
     const int lane = threadIdx.x & 31;
     jobs = jobs_;
     n_jobs = n_jobs_;
     wi = wi_;
-    nw = nw_;
     n = 0;
     my_ring = ring + (size_t)(threadIdx.x >> 5) * kStages * kVpl * 32 + lane;
     my_ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(my_ring));
-    in = Cursor{0, -1};
-    advance(in, jobs, n_jobs, wi, nw);
+    const int c0 = (int)((long long)chunks * wi / nw);
+    const int c1 = (int)((long long)chunks * (wi + 1) / nw);
+    in = seek(jobs, n_jobs, c0, c1 - c0);
     out = in;
   }
-  // copies of the segment at `in` into stage st, then the next segment
+  // copies of the next segment at `in` into stage st
   __device__ void issue(int st) {
     const int lane = threadIdx.x & 31;
-    if (in.j < n_jobs) {
+    const int nq = min(kVpl, in.left);
+    for (int q = 0; q < nq;) {
       const RowJob& jb = jobs[in.j];
-      const int spr = job_spr(jb), nvec = jb.L / 8;
-      const int row = jb.r0 + wi + nw * (in.k / spr);
-      const uint4* wr = reinterpret_cast<const uint4*>(jb.w + (size_t)row * jb.L);
-      const int v0 = (in.k % spr) * 32 * kVpl + lane;
-#pragma unroll
-      for (int q = 0; q < kVpl; ++q)
-        if (v0 + 32 * q < nvec)
-          cp_async16(my_ring_s + (uint32_t)((st * kVpl + q) * 32 * 16), wr + v0 + 32 * q);
-      advance(in, jobs, n_jobs, wi, nw);
+      const int cpr = jb.cpr;
+      const int run = min(nq - q, cpr - in.cc);
+      const int v0 = in.cc * 32 + lane;
+      const uint4* src =
+          reinterpret_cast<const uint4*>(jb.w + (size_t)(jb.r0 + in.row) * jb.L) + v0;
+      const int vleft = jb.nvec - v0;   // vectors of the row from this lane's first on
+      uint32_t dst = my_ring_s + (uint32_t)((st * kVpl + q) * 32 * 16);
+      for (int i = 0; i < run; ++i, dst += 32 * 16)
+        if (32 * i < vleft) cp_async16(dst, src + 32 * i);
+      q += run;
+      step(in, jobs, n_jobs, run, cpr, jb.r1 - jb.r0);
     }
     cp_async_commit();   // (an empty group at the end keeps the wait count uniform)
   }
@@ -301,41 +337,117 @@ struct JobStream {
     for (int st = 0; st < kStages - 1; ++st) issue(st);
   }
   template <int kA>
-  __device__ void run(const Params& p, const uint4* stage, float* ycache, float* scache) {
+  __device__ void run(const Params& p, const uint4* stage, float* ycache, float* scache,
+                      Partial* part) {
     const int lane = threadIdx.x & 31;
-    float acc[kA][2];
+    float acc0[kA], acc1[kA];
 #pragma unroll
-    for (int a = 0; a < kA; ++a) acc[a][0] = acc[a][1] = 0.f;
-    for (; out.j < n_jobs; ++n) {
+    for (int a = 0; a < kA; ++a) acc0[a] = acc1[a] = 0.f;
+    bool head = out.cc == 0;   // the current row's first chunk is in this range
+    int slot = 0;              // partial slot of the next row finished here
+    while (out.left > 0) {
       issue((n + kStages - 1) % kStages);
       asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 1) : "memory");   // segment n landed
-      const RowJob& jb = jobs[out.j];
-      const int spr = job_spr(jb), nvec = jb.L / 8;
-      const int v0 = (out.k % spr) * 32 * kVpl + lane;
       const uint4* buf = my_ring + (size_t)(n % kStages) * kVpl * 32;
+      const int nq = min(kVpl, out.left);
+      for (int q = 0; q < nq;) {
+        const RowJob& jb = jobs[out.j];
+        const int cpr = jb.cpr, A = jb.A;
+        const int run = min(nq - q, cpr - out.cc);
+        const int v0 = out.cc * 32 + lane;
+        const int vleft = jb.nvec - v0;
+        const uint4* w = buf + q * 32;
+        const uint4* x[kA];
 #pragma unroll
-      for (int q = 0; q < kVpl; ++q) {
-        if (v0 + 32 * q < nvec) {
-          const uint4 wv = buf[q * 32];
+        for (int a = 0; a < kA; ++a) x[a] = stage + jb.act[a] + v0;
+        int i = 0;
+        for (; i + 1 < run; i += 2) {
+          if (32 * i < vleft) {
+            const uint4 wv = w[32 * i];
+#pragma unroll
+            for (int a = 0; a < kA; ++a)
+              if (a < A) acc0[a] = dot8(wv, x[a][32 * i], acc0[a]);
+          }
+          if (32 * (i + 1) < vleft) {
+            const uint4 wv = w[32 * (i + 1)];
+#pragma unroll
+            for (int a = 0; a < kA; ++a)
+              if (a < A) acc1[a] = dot8(wv, x[a][32 * (i + 1)], acc1[a]);
+          }
+        }
+        if (i < run && 32 * i < vleft) {
+          const uint4 wv = w[32 * i];
 #pragma unroll
           for (int a = 0; a < kA; ++a)
-            if (a < jb.A) acc[a][q & 1] = dot8(wv, stage[jb.act[a] + v0 + 32 * q], acc[a][q & 1]);
+            if (a < A) acc0[a] = dot8(wv, x[a][32 * i], acc0[a]);
         }
-      }
-      if (out.k % spr == spr - 1) {   // the row's last segment
-        float sum[kA];
+        q += run;
+        const bool tail = out.cc + run == cpr;
+        if (tail || out.left == run) {   // the row ends here, or the range does
+          float sum[kA];
 #pragma unroll
-        for (int a = 0; a < kA; ++a) {
-          sum[a] = acc[a][0] + acc[a][1];
-          acc[a][0] = acc[a][1] = 0.f;
+          for (int a = 0; a < kA; ++a) {
+            sum[a] = acc0[a] + acc1[a];
+            acc0[a] = acc1[a] = 0.f;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int a = 0; a < kA; ++a) sum[a] += __shfl_xor_sync(0xffffffffu, sum[a], o);
+          float mine = sum[0];
+#pragma unroll
+          for (int a = 1; a < kA; ++a)
+            if (lane == a) mine = sum[a];
+          if (head && tail) {
+            if (lane < A) emit(jb, p, jb.r0 + out.row, lane, mine, ycache, scache);
+          } else {
+            Partial& pt = part[2 * wi + slot];
+            if (lane < kDecodeMaxT) pt.v[lane] = mine;
+            if (lane == 0) {
+              pt.valid = 1;
+              pt.head = head ? 1 : 0;
+              pt.tail = tail ? 1 : 0;
+              pt.job = out.j;
+              pt.row = out.row;
+            }
+          }
+          slot = 1;
+          head = true;
         }
-        row_out<kA>(jb, p, jb.r0 + wi + nw * (out.k / spr), sum, ycache, scache);
+        step(out, jobs, n_jobs, run, cpr, jb.r1 - jb.r0);
       }
-      advance(out, jobs, n_jobs, wi, nw);
+      ++n;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   }
 };
+
+// Rows cut by the warp boundaries of a phase (nw warps): the part holding a
+// row's first chunk adds the parts of the following warps in warp order and
+// emits the row. Called by all threads after the phase's parts are visible
+// (a __syncthreads); each row is finished by one thread.
+__device__ void finish_cut_rows(const RowJob* jobs, const Partial* part, int nw, const Params& p,
+                                float* ycache, float* scache) {
+  const int i = threadIdx.x;
+  if (i >= 2 * nw) return;
+  const Partial& h = part[i];
+  if (!h.valid || !h.head) return;
+  float v[kDecodeMaxT];
+#pragma unroll
+  for (int a = 0; a < kDecodeMaxT; ++a) v[a] = h.v[a];
+  bool done = h.tail != 0;
+  for (int w = (i >> 1) + 1; w < nw && !done; ++w) {
+    const Partial& c = part[2 * w];   // the row goes on as the next range's first row
+    if (!c.valid) continue;           // (a warp with an empty range)
+#pragma unroll
+    for (int a = 0; a < kDecodeMaxT; ++a) v[a] += c.v[a];
+    done = c.tail != 0;
+  }
+  const RowJob& jb = jobs[h.job];
+#pragma unroll
+  for (int a = 0; a < kDecodeMaxT; ++a)
+    if (a < jb.A) emit(jb, p, jb.r0 + h.row, a, v[a], ycache, scache);
+}
 
 // Top-K selection and dispatch of the T <= 4 tokens by one warp, into shared
 // memory; CTA 0 also writes the routing outputs.
@@ -424,9 +536,13 @@ __device__ void route(Smem& s, const Params& p, const float* bias, const float* 
 struct Jobs {
   RowJob router;            // this CTA's W_r rows
   RowJob shared1;           // this CTA's Ws1 rows
-  RowJob g1[kMaxJobs];      // the routed experts' W1 rows of this CTA
+  RowJob g1[kMaxG1Jobs];    // the routed experts' W1 rows of this CTA
   RowJob g2[kMaxJobs];      // this CTA's output columns of each touched W2, then of Ws2
   int n_g1, n_g2;
+  int c_router, c_shared1, c_g1, c_g2;   // chunks of each phase's jobs
+  // rows cut between warps: [0] the shared expert's first layer, [1] the
+  // routed first layer, then (after grid barrier 2) the second layer
+  Partial part[2][2 * kWarps];
 };
 
 // Lists the first- and second-layer jobs of this CTA once the routing is in
@@ -441,6 +557,10 @@ __device__ void list_jobs(const Smem& s, Jobs& J, const Params& p, int h0, int h
   for (int j = 0; j < ns; ++j) {
     const int lo = max(a, j * p.D), hi = min(b, (j + 1) * p.D);
     if (lo >= hi) continue;
+    if (n == kMaxG1Jobs) {   // never with at least kMinCtas CTAs (above)
+      atomicOr(&p.hdr->status, kStatusBadIndex);
+      break;
+    }
     RowJob jb{};
     jb.w = p.w1 + (size_t)s.seg_e[j] * p.D * H;
     jb.r0 = lo - j * p.D;
@@ -482,6 +602,8 @@ __device__ void list_jobs(const Smem& s, Jobs& J, const Params& p, int h0, int h
     J.g2[n++] = jb;
   }
   J.n_g2 = n;
+  J.c_g1 = number_chunks(J.g1, J.n_g1);
+  J.c_g2 = number_chunks(J.g2, J.n_g2);
 }
 
 template <int kA, int kStages>
@@ -525,7 +647,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_forward(const Params p) {
     share(p.Ds, cta, G, &jb.r0, &jb.r1);
     jb.out = kHs;
     J.shared1 = jb;
+    J.c_router = number_chunks(&J.router, 1);
+    J.c_shared1 = p.Ds > 0 ? number_chunks(&J.shared1, 1) : 0;
   }
+  for (int i = tid; i < 2 * 2 * kWarps; i += kThreads) (&J.part[0][0])[i].valid = 0;
   // x (every token), the bias and the noise first, while nothing else is in
   // flight
   for (int v = tid; v < T * H / 8; v += kThreads)
@@ -539,15 +664,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_forward(const Params p) {
   // rows are requested first, so they are at the head of the memory queues
   JobStream<kStages> js;
   if (warp == 0) {
-    js.init(&J.router, 1, 0, 1, ring);
+    js.init(&J.router, 1, J.c_router, 0, 1, ring);
     js.prime();
   }
   __syncthreads();
   if (warp != 0) {
-    js.init(&J.shared1, p.Ds > 0 ? 1 : 0, warp - 1, kWarps - 1, ring);
+    js.init(&J.shared1, 1, J.c_shared1, warp - 1, kWarps - 1, ring);
     js.prime();
   }
-  js.template run<kA>(p, stage, nullptr, nullptr);
+  // (warp 0 streams its whole router job, so it never cuts a row)
+  js.template run<kA>(p, stage, nullptr, nullptr, J.part[0]);
   if (warp == 0) {
     // grid barrier 1 (one arrival per CTA, after this warp's logit stores),
     // then the routing and the job lists of both layers
@@ -568,15 +694,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_forward(const Params p) {
   JobStream<kStages> js2;
   if (!s.abort_flag) {
     ld_acquire(ctr);
-    js.init(J.g1, J.n_g1, warp, kWarps, ring);
+    js.init(J.g1, J.n_g1, J.c_g1, warp, kWarps, ring);
     js.prime();
-    js.template run<kA>(p, stage, nullptr, nullptr);
+    js.template run<kA>(p, stage, nullptr, nullptr, J.part[1]);
     // the second layer's weights do not depend on the first layer's
     // outputs: they are in flight while grid barrier 2 is pending
-    js2.init(J.g2, J.n_g2, warp, kWarps, ring);
+    js2.init(J.g2, J.n_g2, J.c_g2, warp, kWarps, ring);
     js2.prime();
   }
+  __syncthreads();
+  if (!s.abort_flag) {
+    // rows cut between warps: the shared expert's (warps 1-15 of phase 1)
+    // and the routed experts' first layer
+    finish_cut_rows(&J.shared1, J.part[0], kWarps - 1, p, nullptr, nullptr);
+    finish_cut_rows(J.g1, J.part[1], kWarps, p, nullptr, nullptr);
+  }
   grid_arrive(p);   // grid barrier 2: every CTA's Hm and Hs
+  // (every thread has passed the cut-row pass above: the slots are free for
+  // the second layer)
+  if (tid < 2 * kWarps) J.part[1][tid].valid = 0;
   if (tid == 0 && !s.abort_flag) grid_wait(ctr, 2u * (uint32_t)G, s, p);
   __syncthreads();
   if (!s.abort_flag) {
@@ -588,10 +724,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_forward(const Params p) {
                             : __ldcg(reinterpret_cast<const uint4*>(p.hs) + (v - n_hm));
   }
   __syncthreads();
-  if (!s.abort_flag) js2.template run<kA>(p, stage, ycache, scache);
+  if (!s.abort_flag) js2.template run<kA>(p, stage, ycache, scache, J.part[1]);
   // (a CTA that gave up may still have second-layer copies in flight)
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
+  if (!s.abort_flag) {
+    finish_cut_rows(J.g2, J.part[1], kWarps, p, ycache, scache);
+    __syncthreads();
+  }
   if (!s.abort_flag) {
     // combine of this CTA's output columns: y[t, h] = sum_k w[t,k]
     // Yr[inv[t,k], h] (+ S[t, h]), fp32 in k order, one rounding
@@ -661,6 +801,7 @@ static bool decode_device_limits(int* sms, int* smem_max) {
       return false;
     n = v;
     m = w;
+    if (v < dec::kMinCtas) return false;
     cache_sms[dev].store(n, std::memory_order_relaxed);
     cache_smem[dev].store(m, std::memory_order_relaxed);
   }
