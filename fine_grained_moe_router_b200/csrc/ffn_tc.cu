@@ -41,6 +41,12 @@ constexpr int kBM = 128;                        // weight rows per tile (MMA M)
 constexpr int kBK = 64;                         // reduction elements per stage (128 bytes)
 constexpr int kBoxRows = 32;                    // activation rows per TMA box
 constexpr int kBoxBytes = kBoxRows * kBK * 2;   // 4 KB
+// Tiles with more than kWideMin activation rows per CTA load them in boxes
+// of kWideRows: each TMA instruction costs the issuing thread on the order
+// of a hundred cycles whatever its size, so at full MMA rate four 32-row
+// boxes per stage keep the producer busy most of the time.
+constexpr int kWideRows = 128;
+constexpr int kWideMin = 64;
 constexpr int kABytes = kBM * kBK * 2;          // 16 KB
 constexpr int kMaxStages = 12;
 constexpr int kStageArea = 192 * 1024;          // shared memory of the operand ring
@@ -263,6 +269,7 @@ struct Args {
   int dense_rows, dense_m_tiles, dense_splits;
   int dense_mtile;     // weight rows per dense tile: kBM, or 2 * kBM on CTA pairs
   int nbox_max;        // activation boxes per stage (rows per tile <= 32 * nbox_max)
+  int wide;            // 1: the wide-box maps may be used (the stage holds whole wide boxes)
   int stage_bytes;     // kABytes + nbox_max * kBoxBytes
   int n_stages;        // stages in the ring (<= kMaxStages)
   uint32_t* status;
@@ -400,7 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmA1,
-                    const __grid_constant__ CUtensorMap tmB1, const Args args) {
+                    const __grid_constant__ CUtensorMap tmB1,
+                    const __grid_constant__ CUtensorMap tmB0w,
+                    const __grid_constant__ CUtensorMap tmB1w, const Args args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -475,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sd = (tl.g < args.E) ? 0 : 1;
         const Side& S = args.side[sd];
         const CUtensorMap* ma = sd ? &tmA1 : &tmA0;
-        const CUtensorMap* mb = sd ? &tmB1 : &tmB0;
+        const CUtensorMap* mb = sd ? &tmB1 : &tmB0;   // (or the wide-box map, below)
         const int arow = (sd ? 0 : tl.g * S.m_rows) + tl.m0 + (int)rank * kBM;
         int nmma = (tl.n + 15) & ~15;
         if (nmma > n_max) {   // never by construction; keeps the ring in bounds
@@ -484,11 +493,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int rows_here = kPair ? nmma / 2 : nmma;   // activation rows this CTA loads
         const int brow = tl.r0 + (int)rank * rows_here;
-        const int nbox = (rows_here + kBoxRows - 1) / kBoxRows;
+        // wide boxes when the tile has enough rows and the stage holds them
+        // (rows past the tile's, loaded as well, feed no MMA column)
+        const bool wide = args.wide && rows_here > kWideMin;
+        const int box_rows = wide ? kWideRows : kBoxRows;
+        const int nbox = (rows_here + box_rows - 1) / box_rows;
+        if (wide) mb = sd ? &tmB1w : &tmB0w;
         // weight rows actually loaded: 128, or fewer for a gate matrix with
         // E < 128 rows (the other rows of the smem tile only feed outputs
         // that are never stored)
-        const uint32_t bytes_here = (uint32_t)S.a_rows * kBK * 2 + (uint32_t)nbox * kBoxBytes;
+        const uint32_t bytes_here =
+            (uint32_t)S.a_rows * kBK * 2 + (uint32_t)(nbox * box_rows) * kBK * 2;
         const int kb0 = tl.ks * S.kb_per, kb1 = min(S.kb, kb0 + S.kb_per);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, args.status)) {
@@ -504,11 +519,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t fb0 = map_to_rank(fb, 0);
             tma_load_2d_pair(sa, ma, kb * kBK, arow, fb0);
             for (int i = 0; i < nbox; ++i)
-              tma_load_2d_pair(sb + i * kBoxBytes, mb, kb * kBK, brow + i * kBoxRows, fb0);
+              tma_load_2d_pair(sb + i * box_rows * kBK * 2, mb, kb * kBK, brow + i * box_rows, fb0);
           } else {
             tma_load_2d(sa, ma, kb * kBK, arow, fb);
             for (int i = 0; i < nbox; ++i)
-              tma_load_2d(sb + i * kBoxBytes, mb, kb * kBK, brow + i * kBoxRows, fb);
+              tma_load_2d(sb + i * box_rows * kBK * 2, mb, kb * kBK, brow + i * box_rows, fb);
           }
           issued[stage] = true;
           issued_parity[stage] = phase;
@@ -728,7 +743,7 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
   auto a_rows_of = [](const TcProblem& p) {
     return p.w_rows >= (uint64_t)kBM ? kBM : (int)((p.w_rows + 7) & ~7ull);
   };
-  CUtensorMap a0, b0, a1, b1;
+  CUtensorMap a0, b0, a1, b1, b0w, b1w;
   if (!make_map(&a0, routed.w, routed.w_rows, routed.kd, a_rows_of(routed)) ||
       !make_map(&b0, routed.act, routed.act_rows, routed.kd, kBoxRows))
     return cudaErrorInvalidValue;
@@ -772,6 +787,20 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
   const int rows_per_cta = pair ? max_n / 2 : max_n;
   args.nbox_max = std::max(1, (rows_per_cta + kBoxRows - 1) / kBoxRows);
   args.stage_bytes = kABytes + args.nbox_max * kBoxBytes;
+  // Wide boxes where a stage holds a whole number of them and both
+  // activation matrices have at least a wide box of rows.
+  args.wide = ((args.nbox_max * kBoxRows) % kWideRows == 0 &&
+               routed.act_rows >= (uint64_t)kWideRows && sh.act_rows >= (uint64_t)kWideRows)
+                  ? 1
+                  : 0;
+  if (args.wide) {
+    if (!make_map(&b0w, routed.act, routed.act_rows, routed.kd, kWideRows) ||
+        !make_map(&b1w, sh.act, sh.act_rows, sh.kd, kWideRows))
+      return cudaErrorInvalidValue;
+  } else {
+    b0w = b0;
+    b1w = b1;
+  }
   args.n_stages = std::min(kMaxStages, kStageArea / args.stage_bytes);
   args.status = status;
   args.E = E;
@@ -781,11 +810,11 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
   if (!pair) {
     const int grid = dense ? std::min(sms, std::max(1, dense->tiles)) : sms;
     return launch_pdl(grouped_gemm_tc<false>, dim3(grid), dim3(kThreads), kSmemBytes, st, a0, b0,
-                      a1, b1, args);
+                      a1, b1, b0w, b1w, args);
   }
   const int pairs = dense ? std::min(sms / 2, std::max(1, dense->tiles)) : sms / 2;
   return launch_pdl_cluster2(grouped_gemm_tc<true>, dim3(2 * std::max(1, pairs)), dim3(kThreads),
-                             kSmemBytes, st, a0, b0, a1, b1, args);
+                             kSmemBytes, st, a0, b0, a1, b1, b0w, b1w, args);
 }
 
 }  // namespace moe
