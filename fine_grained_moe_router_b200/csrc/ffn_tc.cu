@@ -13,8 +13,12 @@
 //
 // Per CTA (persistent, one per SM, 320 threads):
 //   warp 8  TMA producer: weight slab [128 x 64] + activation rows [n x 64]
-//           per stage into 128-byte-swizzled shared memory; the ring has 4
-//           stages for 256-row tiles and up to 12 when the batch is small
+//           per reduction block into 128-byte-swizzled shared memory; a
+//           prefill-sized CTA pair takes two reduction blocks per stage (one
+//           3D box per operand: each TMA instruction costs the issuing thread
+//           about a hundred cycles, which at full MMA rate made the producer
+//           the bottleneck), smaller launches one per stage and up to 12
+//           stages when the batch is small
 //   warp 9  TMEM allocator and MMA issuer: tcgen05.mma kind::f16 (bf16 in,
 //           fp32 accumulate), two 256-column TMEM accumulators so the
 //           epilogue of one tile overlaps the MMAs of the next
@@ -196,6 +200,17 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t a, uint6
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+// 3D form: a box spanning two consecutive reduction blocks (the map's third
+// dimension steps 64 elements along the rows), written as two K-major tiles
+// one after the other.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, int y,
+                                                 int z, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(z), "r"(bar_cluster)
+      : "memory");
 }
 // Arrive on the barrier at this offset in both CTAs of the pair once every
 // MMA issued so far has completed.
@@ -402,7 +417,9 @@ __device__ __noinline__ void split_fixup(const Args& args, const Tile& tl, const
 // M = 256 issued by the even CTA); each CTA loads its 128 weight rows and half
 // of the tile's activation rows per stage, so an SM streams a third less
 // operand data per MMA cycle than with single-CTA tiles of the same N.
-template <bool kPair>
+// kKpb: reduction blocks per ring stage (2 only on CTA pairs whose weight and
+// activation maps are the 3D two-block maps).
+template <bool kPair, int kKpb>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmB0,
@@ -505,22 +522,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t bytes_here =
             (uint32_t)S.a_rows * kBK * 2 + (uint32_t)(nbox * box_rows) * kBK * 2;
         const int kb0 = tl.ks * S.kb_per, kb1 = min(S.kb, kb0 + S.kb_per);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += kKpb) {
           if (!wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
           }
           const uint32_t fb = smem_u32(&full[stage]);
-          // the leader's barrier counts the bytes of both CTAs
-          if (leader) mbar_expect_tx(fb, (kPair ? 2u : 1u) * bytes_here);
           const uint32_t sa = smem_u32(ring + (size_t)stage * stage_bytes);
           const uint32_t sb = sa + kABytes;
-          if (kPair) {
+          if constexpr (kPair && kKpb == 2) {
+            // two reduction blocks (a last odd block's box reaches into the
+            // next split's or past the matrix's end: loaded, never multiplied)
+            if (leader) mbar_expect_tx(fb, 2u * 2u * 2u * (uint32_t)kABytes);
+            const uint32_t fb0 = map_to_rank(fb, 0);
+            tma_load_3d_pair(sa, ma, arow, kb, fb0);
+            tma_load_3d_pair(sa + 2 * kABytes, sd ? &tmB1w : &tmB0w, brow, kb, fb0);
+          } else if (kPair) {
+            // the leader's barrier counts the bytes of both CTAs
+            if (leader) mbar_expect_tx(fb, 2u * bytes_here);
             const uint32_t fb0 = map_to_rank(fb, 0);
             tma_load_2d_pair(sa, ma, kb * kBK, arow, fb0);
             for (int i = 0; i < nbox; ++i)
               tma_load_2d_pair(sb + i * box_rows * kBK * 2, mb, kb * kBK, brow + i * box_rows, fb0);
           } else {
+            mbar_expect_tx(fb, bytes_here);
             tma_load_2d(sa, ma, kb * kBK, arow, fb);
             for (int i = 0; i < nbox; ++i)
               tma_load_2d(sb + i * box_rows * kBK * 2, mb, kb * kBK, brow + i * box_rows, fb);
@@ -554,22 +579,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bounded(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += kKpb) {
           if (!wait_bounded(smem_u32(&full[stage]), phase, abort_flag, args.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(ring + (size_t)stage * stage_bytes);
-          const uint64_t adesc = sw128_desc(sa);
-          const uint64_t bdesc = sw128_desc(sa + kABytes);
+          // stage layout: kKpb weight tiles, then kKpb activation tiles
+          const uint32_t sb = sa + (uint32_t)(kKpb * kABytes);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {   // 16 elements = 32 bytes per MMA
-            const uint32_t accum = (kb != kb0 || k != 0) ? 1u : 0u;
-            if (kPair)
-              mma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
-            else
-              mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+          for (int j = 0; j < kKpb; ++j) {
+            if (kb + j >= kb1) break;
+            const uint64_t adesc = sw128_desc(sa + j * kABytes);
+            const uint64_t bdesc = sw128_desc(sb + j * kABytes);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {   // 16 elements = 32 bytes per MMA
+              const uint32_t accum = (kb + j != kb0 || k != 0) ? 1u : 0u;
+              if (kPair)
+                mma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+              else
+                mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+            }
           }
           if (kPair)
             mma_commit_pair(smem_u32(&empty[stage]));
@@ -703,6 +734,22 @@ static EncodeTiledFn encode_fn() {
 
 // 2D bf16 map over a row-major [rows, cols] matrix, boxes of 64 columns x
 // box_rows rows, 128-byte swizzle, zero fill outside the matrix.
+// 3D bf16 map over the same matrix: (64 columns, rows, column block of 64)
+// with boxes of 64 x box_rows x 2, i.e. two consecutive reduction blocks of
+// box_rows rows, 128-byte swizzle, zero fill outside the matrix.
+static bool make_map_2kb(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kBK, rows, cols / kBK};
+  cuuint64_t strides[2] = {cols * 2, (cuuint64_t)kBK * 2};
+  cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                      uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -730,10 +777,13 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
-    e = cudaFuncSetAttribute(grouped_gemm_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(grouped_gemm_tc<false, 1>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(grouped_gemm_tc<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(grouped_gemm_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(grouped_gemm_tc<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
@@ -801,6 +851,18 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
     b0w = b0;
     b1w = b1;
   }
+  // Prefill-sized CTA pairs (a full 128-row activation box per CTA and
+  // 128-row weight boxes): two reduction blocks per stage, 3D maps.
+  const bool two_blocks = pair && args.wide && args.nbox_max * kBoxRows == kWideRows &&
+                          a_rows_of(routed) == kBM && a_rows_of(sh) == kBM;
+  if (two_blocks) {
+    args.stage_bytes = 2 * (kABytes + kWideRows * kBK * 2);
+    if (!make_map_2kb(&a0, routed.w, routed.w_rows, routed.kd, kBM) ||
+        !make_map_2kb(&a1, sh.w, sh.w_rows, sh.kd, kBM) ||
+        !make_map_2kb(&b0w, routed.act, routed.act_rows, routed.kd, kWideRows) ||
+        !make_map_2kb(&b1w, sh.act, sh.act_rows, sh.kd, kWideRows))
+      return cudaErrorInvalidValue;
+  }
   args.n_stages = std::min(kMaxStages, kStageArea / args.stage_bytes);
   args.status = status;
   args.E = E;
@@ -809,11 +871,14 @@ cudaError_t launch_grouped_gemm_tc(const TcProblem& routed, const TcProblem& sha
   const int sms = (max_ctas > 0) ? std::min(num_sms, max_ctas) : num_sms;
   if (!pair) {
     const int grid = dense ? std::min(sms, std::max(1, dense->tiles)) : sms;
-    return launch_pdl(grouped_gemm_tc<false>, dim3(grid), dim3(kThreads), kSmemBytes, st, a0, b0,
-                      a1, b1, b0w, b1w, args);
+    return launch_pdl(grouped_gemm_tc<false, 1>, dim3(grid), dim3(kThreads), kSmemBytes, st, a0,
+                      b0, a1, b1, b0w, b1w, args);
   }
   const int pairs = dense ? std::min(sms / 2, std::max(1, dense->tiles)) : sms / 2;
-  return launch_pdl_cluster2(grouped_gemm_tc<true>, dim3(2 * std::max(1, pairs)), dim3(kThreads),
+  if (two_blocks)
+    return launch_pdl_cluster2(grouped_gemm_tc<true, 2>, dim3(2 * std::max(1, pairs)),
+                               dim3(kThreads), kSmemBytes, st, a0, b0, a1, b1, b0w, b1w, args);
+  return launch_pdl_cluster2(grouped_gemm_tc<true, 1>, dim3(2 * std::max(1, pairs)), dim3(kThreads),
                              kSmemBytes, st, a0, b0, a1, b1, b0w, b1w, args);
 }
 
