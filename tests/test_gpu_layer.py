@@ -108,6 +108,17 @@ def test_layer_edge_shapes(M, dtype, E, K, Ds):
         run_and_check(M, L, T)
 
 
+# CTA-pair layers (two reduction blocks per ring stage) whose second layer
+# splits its reduction into an odd number of blocks per split (24 blocks as
+# 5+5+5+5+4, or 24 over 5 at T = 384): the box of a split's last stage
+# reaches into the next split's first block, which must not be multiplied.
+@pytest.mark.parametrize("T,H,E,K,D,Ds", [(256, 768, 4, 2, 1536, 768), (384, 512, 4, 4, 1536, 512)])
+def test_layer_pair_odd_blocks_per_split(M, T, H, E, K, D, Ds):
+    wl = mi.Workload("pairsplit", "CTA pairs, odd reduction blocks per split", "bf16", H, E, K, D,
+                     Ds, (T,), 23, zipf_s=0.8)
+    run_and_check(M, DeviceLayer(wl), T)
+
+
 def test_layer_empty_batch_is_a_no_op(M):
     L = layer("c1")
     d = L.desc(M, 0)
