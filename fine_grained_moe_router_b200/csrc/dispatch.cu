@@ -138,6 +138,7 @@ __device__ __forceinline__ void tc_row_split(int c, int* nt, int* rows) {
   *rows = r;
 }
 
+constexpr int kFlatTileList = 8192;   // tiles above which every thread shares the writing
 
 // Writes the tile lists of every group; thread e < E owns expert e (c rows
 // starting at row `off`), thread E owns the shared expert (T token rows).
@@ -215,65 +216,62 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
   }
   __syncthreads();
   if (ts.tc1) {
-    // The two lists as one index space (list 1, then list 2), cut into one
-    // contiguous range per thread. A thread locates its first tile once
-    // (group by binary search over the rank positions, then the tile's
-    // place in its group) and walks on from there: the next tile's row
-    // block, weight block and split follow from the current one without a
-    // division, and a group's end moves to the next non-empty group. (A
-    // division or search per tile made the list's writing instruction-bound
-    // on the one SM: ~16 us for 12k tiles.)
-    const int n1_all = sh1 + tot1, n2_all = sh2 + tot2, n_all = n1_all + n2_all;
-    const int per = (n_all + (int)blockDim.x - 1) / (int)blockDim.x;
-    int i = (int)threadIdx.x * per;
-    const int i_end = min(n_all, i + per);
-    if (i < i_end) {
-      int list = i < n1_all ? 0 : 1;
-      int rank, j;   // rank -1: the shared expert's group
-      {
-        const int li = list ? i - n1_all : i;   // position in its list
-        const int shn = list ? sh2 : sh1;
-        if (li < shn) {
-          rank = -1;
-          j = li;
-        } else {
-          const int k = li - shn;
-          const int* pos = list ? s_pos2 : s_pos1;
-          int lo = 0, hi = E - 1;   // last rank position with pos <= k (a non-empty group)
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (pos[mid] <= k)
-              lo = mid;
-            else
-              hi = mid - 1;
+    const int n1_all = sh1 + tot1, n2_all = sh2 + tot2;
+    // Long lists (a long batch: thousands of tiles in the shared expert's or
+    // a hot expert's group) are spread over all threads, each finding its
+    // tile's group by binary search over the groups' first positions;
+    // shorter ones go one group per warp, which needs no search.
+    const bool flat = n1_all + n2_all > kFlatTileList;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    int g = flat ? 0 : warp, i_begin = flat ? threadIdx.x : lane;
+    const int i_step = flat ? (int)blockDim.x : 32;
+    while (g <= E) {
+      // tiles of group g (per-warp mode) or of both whole lists (flat mode)
+      const int nt_g = s_nt[g];
+      const int m1_g = (g < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared;
+      const int sp1_g = (g < E) ? ts.splits1_routed : ts.splits1_shared;
+      const int sp2_g = (g < E) ? ts.splits2_routed : ts.splits2_shared;
+      const int n_items = flat ? n1_all + n2_all : nt_g * (m1_g * sp1_g + ts.m_tiles2 * sp2_g);
+      for (int i = i_begin; i < n_items; i += i_step) {
+        int gg = g, j;
+        bool first;
+        if (flat) {
+          first = i < n1_all;
+          const int li = first ? i : i - n1_all;   // position in its list
+          const int shn = first ? sh1 : sh2;
+          if (li < shn) {
+            gg = E;
+            j = li;
+          } else {
+            const int k = li - shn;
+            const int* pos = first ? s_pos1 : s_pos2;
+            int lo = 0, hi = E - 1;   // last rank position with pos <= k (a non-empty group)
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (pos[mid] <= k)
+                lo = mid;
+              else
+                hi = mid - 1;
+            }
+            gg = s_grp[lo];
+            j = k - pos[lo];
           }
-          rank = lo;
-          j = k - pos[lo];
+        } else {
+          const int n1 = nt_g * m1_g * sp1_g;
+          first = i < n1;
+          j = first ? i : i - n1;
         }
-      }
-      // geometry of the current group
-      int gg, nt, mt, sp, size, first_pos;
-      bool row_outer;
-      auto enter = [&]() {
-        gg = rank < 0 ? E : s_grp[rank];
-        nt = s_nt[gg];
-        mt = list == 0 ? (gg < E ? ts.m_tiles1_routed : ts.m_tiles1_shared) : ts.m_tiles2;
-        sp = list == 0 ? (gg < E ? ts.splits1_routed : ts.splits1_shared)
-                       : (gg < E ? ts.splits2_routed : ts.splits2_shared);
-        size = nt * mt * sp;
-        // Order inside the group: when the group has more activation rows
-        // than weight rows the row blocks are outermost (the weight matrix
-        // stays in L2 while the rows stream once); otherwise the weight
-        // blocks are outermost (each weight slab streams once while its row
-        // blocks, on neighbouring CTAs, reuse it from L2). Splits vary
-        // fastest after that.
-        row_outer = s_rows[gg] > mt * ts.mtile;
-        first_pos = list == 0 ? s_first1[gg] : s_first2[gg];
-      };
-      enter();
-      int r, mb, ks;   // row block, weight block, split of tile j
-      {
-        int q;
+        const int nt = s_nt[gg];
+        const int sp = first ? ((gg < E) ? ts.splits1_routed : ts.splits1_shared)
+                             : ((gg < E) ? ts.splits2_routed : ts.splits2_shared);
+        const int mt = first ? ((gg < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared) : ts.m_tiles2;
+        // Order inside the group: when the group has more activation rows than
+        // weight rows the row blocks are outermost (the weight matrix stays in
+        // L2 while the rows stream once); otherwise the weight blocks are
+        // outermost (each weight slab streams once while its row blocks, on
+        // neighbouring CTAs, reuse it from L2). Splits vary fastest after that.
+        int r, q, j0;   // j0: the position of the split-0 tile of j in the group
+        const bool row_outer = s_rows[gg] > mt * ts.mtile;
         if (row_outer) {
           r = j / (mt * sp);
           q = j - r * (mt * sp);
@@ -281,49 +279,25 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
           r = j % nt;
           q = j / nt;
         }
-        mb = q / sp;
-        ks = q - mb * sp;
-      }
-      for (; i < i_end; ++i) {
         Tile t;
         t.g = gg;
         t.r0 = s_rbase[gg] + r * s_rper[gg];
         t.n = min(s_rper[gg], s_rows[gg] - r * s_rper[gg]);
-        t.m0 = mb * ts.mtile;
-        t.ks = ks;
+        t.m0 = (q / sp) * ts.mtile;
+        t.ks = q % sp;
+        j0 = row_outer ? j - t.ks : j - t.ks * nt;
         t.arrivals[0] = 0;
         t.arrivals[1] = 0;
-        t.first_split = first_pos + (row_outer ? j - ks : j - ks * nt);   // its split-0 tile
-        (list == 0 ? ts.tc1 : ts.tc2)[first_pos + j] = t;
-        // the next tile
-        if (++j == size) {
-          // the next non-empty group of this list, else the start of list 2
-          j = r = mb = ks = 0;
-          do {
-            if (rank + 1 < E) {
-              ++rank;
-            } else {
-              list = 1;
-              rank = sh2 > 0 ? -1 : 0;
-            }
-            enter();
-          } while (size == 0 && !(list == 1 && rank == E - 1));
-        } else if (row_outer) {
-          if (++ks == sp) {
-            ks = 0;
-            if (++mb == mt) {
-              mb = 0;
-              ++r;
-            }
-          }
-        } else if (++r == nt) {
-          r = 0;
-          if (++ks == sp) {
-            ks = 0;
-            ++mb;
-          }
+        if (first) {
+          t.first_split = s_first1[gg] + j0;
+          ts.tc1[s_first1[gg] + j] = t;
+        } else {
+          t.first_split = s_first2[gg] + j0;
+          ts.tc2[s_first2[gg] + j] = t;
         }
       }
+      if (flat) break;
+      g += nwarps;
     }
   }
   if (threadIdx.x == 0) {
