@@ -14,7 +14,12 @@ namespace moe {
 constexpr int kMaxK = 16;
 constexpr int kMaxE = 512;
 constexpr int kForwardEvents = 6;   // stage events of moe_layer_forward_profiled
-constexpr int kDecodeMaxT = 4;      // tokens of the single-launch decode forward (at most)
+// Tokens of the single-launch decode forward (at most). Measured on B200 at
+// the 128- and 256-expert layers: 1 and 2 tokens run faster in one launch
+// than on the multi-launch path (60.6 vs 77.1 us, 98.1 vs 107.5 us), 3 tokens
+// slower (145.8 vs 122.1 us): their staged activations leave the weight
+// rings two stages deep while the tensor-core GEMMs keep streaming.
+constexpr int kDecodeMaxT = 2;
 
 // Status bits written by kernels into the workspace header.
 constexpr uint32_t kStatusTimeout = 1u;

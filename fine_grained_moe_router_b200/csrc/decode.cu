@@ -1,6 +1,6 @@
 // Single-launch forward of a bf16 MoE layer for a handful of tokens (decode).
 //
-// With T <= 4 tokens every expert GEMM of the layer is a matrix-vector
+// With T <= 2 tokens every expert GEMM of the layer is a matrix-vector
 // product against at most four activation rows: the step is bound by the
 // weight bytes it streams from HBM ("Kimi K3 fine-grained MoE under high
 // concurrency", section "通信-计算时间比的代数拐点": 2*H*D multiply-adds per
@@ -54,7 +54,7 @@ namespace dec {
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxRowLen = 16384;                    // elements of the longest weight row
-constexpr int kMaxCopies = kDecodeMaxT * kMaxK;      // 64
+constexpr int kMaxCopies = kDecodeMaxT * kMaxK;      // 32
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
 struct Params {
@@ -449,7 +449,7 @@ __device__ void finish_cut_rows(const RowJob* jobs, const Partial* part, int nw,
     if (a < jb.A) emit(jb, p, jb.r0 + h.row, a, v[a], ycache, scache);
 }
 
-// Top-K selection and dispatch of the T <= 4 tokens by one warp, into shared
+// Top-K selection and dispatch of the T <= 2 tokens by one warp, into shared
 // memory; CTA 0 also writes the routing outputs.
 __device__ void route(Smem& s, const Params& p, const float* bias, const float* noise) {
   const int lane = threadIdx.x & 31;
@@ -853,15 +853,15 @@ cudaError_t launch_decode_forward(const moe_layer_desc& d, const DecodeBuffers& 
   p.D = d.D;
   p.Ds = d.Ds;
   p.h_rows = l.h_rows;
-  // instantiations by activation rows (1, 2, up to 4) and pipeline depth (3, 2)
-  void (*const kernels[3][2])(const Params) = {
+  // instantiations by activation rows (1, 2) and pipeline depth (3, 2)
+  void (*const kernels[2][2])(const Params) = {
       {decode_forward<1, 3>, decode_forward<1, 2>},
-      {decode_forward<2, 3>, decode_forward<2, 2>},
-      {decode_forward<4, 3>, decode_forward<4, 2>}};
-  const int which = d.T == 1 ? 0 : (d.T == 2 ? 1 : 2);
+      {decode_forward<2, 3>, decode_forward<2, 2>}};
+  static_assert(kDecodeMaxT == 2, "one instantiation per token count");
+  const int which = d.T == 1 ? 0 : 1;
   const int deep = l.stages == 3 ? 0 : 1;
   void (*kern)(const Params) = kernels[which][deep];
-  static std::atomic<bool> attr_set[64][3][2];
+  static std::atomic<bool> attr_set[64][2][2];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
