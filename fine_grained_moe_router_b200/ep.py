@@ -23,8 +23,11 @@ rank's T local tokens:
 5. the outputs go back to receive order (moe_gather_rows) and to their
    sources (All-to-All with the splits swapped), arriving in the source's
    dispatch order;
-6. the source computes the shared expert on its tokens and combines
-   (moe_combine): y[t] = sum_k w[t,k] Yr[inv[t,k]] + S[t].
+6. the source combines (moe_combine): y[t] = sum_k w[t,k] Yr[inv[t,k]] +
+   S[t], with S[t] the shared expert's output on its own tokens, computed
+   while the dispatched rows are in flight (step 3 runs asynchronously: the
+   exchange overlaps that compute, the "communication masking" of the Kimi
+   K3 page's section "工业级细粒度 MoE 路由与通信掩盖实战").
 
 Every step of the arithmetic runs in libmoe's kernels through the C ABI;
 torch.distributed carries the exchanges (NCCL over NVLink on GPUs: every
@@ -159,11 +162,20 @@ class ExpertParallelMoE:
         dist.all_to_all_single(recv_counts, send_counts, group=self.group)
         send_splits = send_counts.sum(dim=1).tolist()
         recv_splits = recv_counts.sum(dim=1).tolist()
-        # 3. the dispatched rows to the owners
+        # 3. the dispatched rows to the owners, in flight while the shared
+        #    expert runs on this rank's tokens
         send_rows = ops.gather_rows(x, perm, K)
         recv_rows = torch.empty((sum(recv_splits), self.H), dtype=x.dtype, device=x.device)
-        dist.all_to_all_single(recv_rows, send_rows, output_split_sizes=recv_splits,
-                               input_split_sizes=send_splits, group=self.group)
+        exchange = dist.all_to_all_single(recv_rows, send_rows, output_split_sizes=recv_splits,
+                                          input_split_sizes=send_splits, group=self.group,
+                                          async_op=True)
+        y_shared = None
+        if self.ws1 is not None:
+            T = x.shape[0]
+            tok = torch.arange(T, dtype=torch.int32, device=x.device)
+            one = torch.tensor([0, T], dtype=torch.int32, device=x.device)
+            y_shared = ops.experts(x, tok, one, self.ws1.unsqueeze(0), self.ws2.unsqueeze(0))
+        exchange.wait()
         # 4. this rank's experts over the received rows, expert by expert
         loc_off, loc_perm, loc_inv = ops.local_order(recv_counts)
         y_local = ops.experts(recv_rows, loc_perm, loc_off, self.w1, self.w2)
@@ -172,13 +184,7 @@ class ExpertParallelMoE:
         y_rows = torch.empty((perm.numel(), self.H), dtype=y_back.dtype, device=x.device)
         dist.all_to_all_single(y_rows, y_back, output_split_sizes=send_splits,
                                input_split_sizes=recv_splits, group=self.group)
-        # 6. shared expert on the local tokens, combine
-        y_shared = None
-        if self.ws1 is not None:
-            T = x.shape[0]
-            tok = torch.arange(T, dtype=torch.int32, device=x.device)
-            one = torch.tensor([0, T], dtype=torch.int32, device=x.device)
-            y_shared = ops.experts(x, tok, one, self.ws1.unsqueeze(0), self.ws2.unsqueeze(0))
+        # 6. combine with the shared expert's output
         y = ops.combine(y_rows, w, inv, y_shared, x.dtype)
         if routing is not None:
             routing.update(logits=logits, topk_idx=idx, topk_w=w, counts=counts,
