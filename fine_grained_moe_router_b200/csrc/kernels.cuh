@@ -77,8 +77,12 @@ cudaError_t launch_dispatch_scratch(const moe_layer_desc& d, int n_chunks, int32
                                    int32_t* inv, cudaStream_t st);
 cudaError_t launch_tiles_from_offsets(const moe_layer_desc& d, const WsLayout& L, char* ws,
                                       const int32_t* offsets, bool tc_tiles, cudaStream_t st);
+// xp[row] = x[perm[row] / K]; with inv (from the same dispatch) and at least
+// kGatherByTokenMinT tokens the copy is walked by token (each x row read once).
+constexpr int kGatherByTokenMinT = 2048;
 cudaError_t launch_gather_rows(const moe_layer_desc& d, const void* x, const int32_t* perm,
-                               void* xp, int num_sms, cudaStream_t st);
+                               void* xp, int num_sms, cudaStream_t st,
+                               const int32_t* inv = nullptr);
 // dst[r] = src[idx[r] / divisor] (row_vecs 16-byte vectors a row) for r < n_rows; idx
 // values at or above idx_bound (or negative) leave the row unwritten.
 cudaError_t launch_gather_rows_raw(const void* src, int idx_bound, const int32_t* idx, int n_rows,

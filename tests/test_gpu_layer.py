@@ -135,3 +135,25 @@ def test_workspace_too_small_is_rejected(M):
     with pytest.raises(M.MoEError) as ei:
         M.moe_layer_forward(d, L.weights(M), x, torch.empty_like(x), None, small)
     assert ei.value.status == 3
+
+
+# The benchmark times the expert GEMMs alone by re-running them on what the
+# last forward left in the workspace (moe_expert_gemms): recomputing the same
+# first-layer outputs and expert outputs must leave the workspace bit for bit
+# as the forward left it, on CTA pairs (c2 T=512) and single-CTA tiles (c3 T=16).
+@pytest.mark.parametrize("key,T", [("c2", 512), ("c3", 16)])
+def test_expert_gemms_recompute_the_forward_bit_for_bit(M, key, T):
+    L = layer(key)
+    wl = L.wl
+    x = mi.draw_x(wl, T).cuda()
+    d = L.desc(M, T)
+    ws = M.alloc_workspace(d)
+    y = torch.empty_like(x)
+    M.moe_layer_forward(d, L.weights(M), x, y, None, ws)
+    torch.cuda.synchronize()
+    before = ws.clone()
+    M.moe_expert_gemms(d, L.weights(M), x, ws)
+    torch.cuda.synchronize()
+    assert M.moe_check_status(ws) == 0
+    # (moe_check_status clears the status word, which was zero before)
+    assert torch.equal(ws, before)
