@@ -121,6 +121,8 @@ struct TileSpec {
   int splits2_routed, splits2_shared;     // reduction splits of GEMM2 tiles
   int mtile;                              // weight rows per tile: 128, or 256 on CTA pairs
   int lpt;                                // 1: experts by descending rows; 0: by index
+  int tc_sliced;                          // 1: the tensor-core lists are written by
+                                          // emit_tiles_sliced after the dispatch kernels
 };
 
 // Number of balanced row tiles for a group of c rows and the rows per tile
@@ -142,26 +144,11 @@ constexpr int kFlatTileList = 8192;   // tiles above which every thread shares t
 
 // Writes the tile lists of every group; thread e < E owns expert e (c rows
 // starting at row `off`), thread E owns the shared expert (T token rows).
-__device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const TileSpec& ts,
-                           int* sh, WsHeader* hdr) {
+// The tensor-core tile lists of emit_tiles (this CTA's slice of them).
+__device__ void emit_tc_tiles(int c, int off, int E, int T, int has_shared, const TileSpec& ts,
+                              int* sh, WsHeader* hdr, int g_rows, int r_base, int slice,
+                              int n_slices) {
   const int e = threadIdx.x;
-  // SIMT tiles: ceil(rows / kSimtRows) row blocks per group.
-  const int g_rows = (e < E) ? c : ((e == E && has_shared) ? T : 0);
-  const int r_base = (e < E) ? off : 0;
-  const int nt_simt = (g_rows + kSimtRows - 1) / kSimtRows;
-  int tot_simt = 0, first_simt = 0;
-  if (ts.simt) first_simt = block_exclusive_scan(nt_simt, sh, &tot_simt);   // uniform branch
-  if (ts.simt) {
-    for (int i = 0; i < nt_simt; ++i) {
-      Tile t;
-      t.g = e;
-      t.r0 = r_base + i * kSimtRows;
-      t.n = min(kSimtRows, g_rows - i * kSimtRows);
-      t.m0 = 0;
-      t.ks = 0;
-      ts.simt[first_simt + i] = t;
-    }
-  }
   // Tensor-core tiles: balanced row blocks (<= kTcRows rows, multiple of 16)
   // times weight-row blocks (128, or 256 on CTA pairs) times reduction
   // splits. Order: the shared expert first, then the routed experts by
@@ -221,9 +208,11 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
     // a hot expert's group) are spread over all threads, each finding its
     // tile's group by binary search over the groups' first positions;
     // shorter ones go one group per warp, which needs no search.
-    const bool flat = n1_all + n2_all > kFlatTileList;
+    const bool flat = n_slices > 1 || n1_all + n2_all > kFlatTileList;
+    const int lo = (int)((long long)(n1_all + n2_all) * slice / n_slices);
+    const int hi = (int)((long long)(n1_all + n2_all) * (slice + 1) / n_slices);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-    int g = flat ? 0 : warp, i_begin = flat ? threadIdx.x : lane;
+    int g = flat ? 0 : warp, i_begin = flat ? lo + (int)threadIdx.x : lane;
     const int i_step = flat ? (int)blockDim.x : 32;
     while (g <= E) {
       // tiles of group g (per-warp mode) or of both whole lists (flat mode)
@@ -231,7 +220,7 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
       const int m1_g = (g < E) ? ts.m_tiles1_routed : ts.m_tiles1_shared;
       const int sp1_g = (g < E) ? ts.splits1_routed : ts.splits1_shared;
       const int sp2_g = (g < E) ? ts.splits2_routed : ts.splits2_shared;
-      const int n_items = flat ? n1_all + n2_all : nt_g * (m1_g * sp1_g + ts.m_tiles2 * sp2_g);
+      const int n_items = flat ? hi : nt_g * (m1_g * sp1_g + ts.m_tiles2 * sp2_g);
       for (int i = i_begin; i < n_items; i += i_step) {
         int gg = g, j;
         bool first;
@@ -300,11 +289,45 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
       g += nwarps;
     }
   }
-  if (threadIdx.x == 0) {
-    hdr->n_tiles[0] = tot_simt;
-    hdr->n_tiles[1] = ts.tc1 ? tot1 + sh1 : 0;
-    hdr->n_tiles[2] = ts.tc1 ? tot2 + sh2 : 0;
+  if (threadIdx.x == 0 && slice == 0) {
+    hdr->n_tiles[1] = tot1 + sh1;
+    hdr->n_tiles[2] = tot2 + sh2;
   }
+}
+
+// slice / n_slices: with n_slices > 1 this CTA writes only its share
+// [n * slice / n_slices, n * (slice + 1) / n_slices) of the n tensor-core
+// tiles (both lists as one index space), slice 0 their counts; n_slices = 0
+// writes no tensor-core tile. The SIMT list is written whole, by slice 0.
+__device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const TileSpec& ts,
+                           int* sh, WsHeader* hdr, int slice = 0, int n_slices = 1) {
+  const int e = threadIdx.x;
+  // SIMT tiles: ceil(rows / kSimtRows) row blocks per group.
+  const int g_rows = (e < E) ? c : ((e == E && has_shared) ? T : 0);
+  const int r_base = (e < E) ? off : 0;
+  const int nt_simt = (g_rows + kSimtRows - 1) / kSimtRows;
+  int tot_simt = 0, first_simt = 0;
+  if (ts.simt) first_simt = block_exclusive_scan(nt_simt, sh, &tot_simt);   // uniform branch
+  if (ts.simt && slice == 0) {
+    for (int i = 0; i < nt_simt; ++i) {
+      Tile t;
+      t.g = e;
+      t.r0 = r_base + i * kSimtRows;
+      t.n = min(kSimtRows, g_rows - i * kSimtRows);
+      t.m0 = 0;
+      t.ks = 0;
+      ts.simt[first_simt + i] = t;
+    }
+  }
+  if (threadIdx.x == 0 && slice == 0) {
+    hdr->n_tiles[0] = tot_simt;
+    if (!ts.tc1) {
+      hdr->n_tiles[1] = 0;
+      hdr->n_tiles[2] = 0;
+    }
+  }
+  if (ts.tc1 && n_slices > 0) emit_tc_tiles(c, off, E, T, has_shared, ts, sh, hdr, g_rows, r_base,
+                                            slice, n_slices);
 }
 
 __global__ void __launch_bounds__(1024) scan_and_tiles(const int32_t* __restrict__ hist,
@@ -348,7 +371,7 @@ __global__ void __launch_bounds__(1024) scan_and_tiles(const int32_t* __restrict
   if (e == E) offsets[E] = total;
   // rows no copy fills (only when some copy had an expert outside [0, E))
   for (int r = total + threadIdx.x; r < TK; r += blockDim.x) perm[r] = -1;
-  emit_tiles(c, off, E, T, has_shared, ts, sh, hdr);
+  emit_tiles(c, off, E, T, has_shared, ts, sh, hdr, 0, ts.tc_sliced ? 0 : 1);
 }
 
 // Tile lists from given offsets (moe_grouped_ffn called on its own).
@@ -366,6 +389,26 @@ __global__ void __launch_bounds__(1024) tiles_from_offsets(const int32_t* __rest
     c = offsets[e + 1] - off;
   }
   emit_tiles(c, off, E, T, has_shared, ts, sh, hdr);
+}
+
+// The tensor-core tile lists from the offsets a dispatch kernel wrote, over
+// many CTAs: each recomputes the groups' table from the offsets and writes
+// its slice of the tiles (one tile per thread or so).
+__global__ void __launch_bounds__(1024) emit_tiles_sliced(const int32_t* __restrict__ offsets,
+                                                          int E, int T, int has_shared,
+                                                          TileSpec ts,
+                                                          WsHeader* __restrict__ hdr) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int sh[96];
+  const int e = threadIdx.x;
+  int c = 0, off = 0;
+  if (e < E) {
+    off = offsets[e];
+    c = offsets[e + 1] - off;
+  }
+  emit_tc_tiles(c, off, E, T, has_shared, ts, sh, hdr, (e < E) ? c : ((e == E && has_shared) ? T : 0),
+                (e < E) ? off : 0, (int)blockIdx.x, (int)gridDim.x);
 }
 
 constexpr int kScatterWarps = 8;
@@ -461,7 +504,7 @@ __device__ void dispatch_block(const int32_t* __restrict__ idx, int TK, int E, i
   }
   if (e == E) offsets[E] = total;
   for (int r = total + threadIdx.x; r < TK; r += blockDim.x) perm[r] = -1;   // unfilled rows
-  emit_tiles(c, off, E, T, has_shared, ts, sh, hdr);
+  emit_tiles(c, off, E, T, has_shared, ts, sh, hdr, 0, ts.tc_sliced ? 0 : 1);
   __syncthreads();
   for (int i0 = w0; i0 < w1; i0 += 32) {
     const int i = i0 + lane;
@@ -619,6 +662,7 @@ static TileSpec make_tile_spec(const moe_layer_desc& d, const WsLayout& L, char*
   ts.tc2 = tc_tiles ? reinterpret_cast<Tile*>(ws + L.tiles_tc2) : nullptr;
   ts.mtile = (split && L.sp.pair) ? 256 : 128;
   ts.lpt = ((long long)d.T * d.K > 4LL * d.E) ? 1 : 0;
+  ts.tc_sliced = 0;
   ts.m_tiles1_routed = d.D / ts.mtile;
   ts.m_tiles1_shared = d.Ds / ts.mtile;
   ts.m_tiles2 = d.H / ts.mtile;
@@ -642,8 +686,20 @@ static cudaError_t dispatch_impl(const moe_layer_desc& d, const WsLayout& L, cha
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
   int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
   const int n_chunks = L.n_chunks;
-  const TileSpec ts = make_tile_spec(d, L, ws, tc_tiles, /*split=*/true);
+  TileSpec ts = make_tile_spec(d, L, ws, tc_tiles, /*split=*/true);
   const int has_shared = (d.Ds > 0 && shared_tiles) ? 1 : 0;
+  // Batches of more than kChunk copies (the three-kernel dispatch): the
+  // tensor-core lists are written over all SMs by a launch of their own,
+  // after the dispatch kernels (which then write only the counts, offsets,
+  // perm and inv); at 16384 tokens of the 128-expert layer, 27 us faster.
+  // Smaller batches keep the one-CTA writing: there the extra launch and the
+  // table every CTA rebuilds cost as much as the writing saves (c3 T=16
+  // 267.5 vs 269.7 us, c4 T=16 275.3 vs 279.5 us, measured).
+  ts.tc_sliced = (tc_tiles && TK > kChunk) ? 1 : 0;
+  auto emit_sliced = [&]() -> cudaError_t {
+    return launch_pdl(emit_tiles_sliced, dim3(num_sms > 0 ? num_sms : 148), dim3(1024), 0, st,
+                      (const int32_t*)offsets, d.E, d.T, has_shared, ts, hdr);
+  };
   if (TK > 0 && TK <= kChunk) {
     // all 32 warps even for a handful of copies: they share the writing of
     // the tile lists (thousands of tiles for a few experts with a wide D)
@@ -663,6 +719,7 @@ static cudaError_t dispatch_impl(const moe_layer_desc& d, const WsLayout& L, cha
                    has_shared, counts, offsets, perm, inv, ts, hdr,
                    static_cast<const uint4*>(fuse_gather ? x : nullptr), d.K, d.H * 2 / 16,
                    static_cast<uint4*>(fuse_gather ? xp : nullptr));
+    if (e == cudaSuccess && ts.tc_sliced) e = emit_sliced();
     if (e != cudaSuccess || fuse_gather || xp == nullptr) return e;
     return launch_gather_rows(d, x, perm, xp, num_sms, st, inv);
   }
@@ -679,6 +736,7 @@ static cudaError_t dispatch_impl(const moe_layer_desc& d, const WsLayout& L, cha
   if (TK > 0)
     e = launch_pdl(chunk_scatter, dim3(n_chunks), dim3(256), 0, st, idx, TK, d.E,
                    (const int32_t*)base, perm, inv);
+  if (e == cudaSuccess && ts.tc_sliced) e = emit_sliced();
   if (e != cudaSuccess || xp == nullptr) return e;
   return launch_gather_rows(d, x, perm, xp, num_sms, st, inv);
 }
