@@ -91,8 +91,8 @@ def algorithmic(wl, T, touched, counts=None):
 # it was measured on: the key is a fingerprint of the GEMM source and the
 # headers it includes with comments and whitespace removed, so any change to
 # the code (not to its comments) makes it null.
-MEASURED_TRAFFIC = {"kernel_code_sha256_16": "2eeca55434c86594", "workload": "c2", "T": 4096,
-                    "bytes_per_step": 1.072410e9 + 0.233183e9 + 1.444714e9 + 0.135630e9}
+MEASURED_TRAFFIC = {"kernel_code_sha256_16": "847c8768f9eabbbe", "workload": "c2", "T": 4096,
+                    "bytes_per_step": 1.106830e9 + 0.234959e9 + 1.445730e9 + 0.135528e9}
 TRAFFIC_SOURCES = ("ffn_tc.cu", "common.cuh", "kernels.cuh")
 
 
