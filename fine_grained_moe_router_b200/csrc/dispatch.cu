@@ -145,9 +145,11 @@ constexpr int kFlatTileList = 8192;   // tiles above which every thread shares t
 // Writes the tile lists of every group; thread e < E owns expert e (c rows
 // starting at row `off`), thread E owns the shared expert (T token rows).
 // The tensor-core tile lists of emit_tiles (this CTA's slice of them).
-__device__ void emit_tc_tiles(int c, int off, int E, int T, int has_shared, const TileSpec& ts,
-                              int* sh, WsHeader* hdr, int g_rows, int r_base, int slice,
-                              int n_slices) {
+// Thread e (one per expert slot, blockDim > E): c rows of expert e; g_rows
+// and r_base the rows and first dispatched row of group e (group E: the
+// shared expert's T rows when present).
+__device__ void emit_tc_tiles(int c, int E, int T, int has_shared, const TileSpec& ts, int* sh,
+                              WsHeader* hdr, int g_rows, int r_base, int slice, int n_slices) {
   const int e = threadIdx.x;
   // Tensor-core tiles: balanced row blocks (<= kTcRows rows, multiple of 16)
   // times weight-row blocks (128, or 256 on CTA pairs) times reduction
@@ -326,8 +328,8 @@ __device__ void emit_tiles(int c, int off, int E, int T, int has_shared, const T
       hdr->n_tiles[2] = 0;
     }
   }
-  if (ts.tc1 && n_slices > 0) emit_tc_tiles(c, off, E, T, has_shared, ts, sh, hdr, g_rows, r_base,
-                                            slice, n_slices);
+  if (ts.tc1 && n_slices > 0)
+    emit_tc_tiles(c, E, T, has_shared, ts, sh, hdr, g_rows, r_base, slice, n_slices);
 }
 
 __global__ void __launch_bounds__(1024) scan_and_tiles(const int32_t* __restrict__ hist,
@@ -407,7 +409,7 @@ __global__ void __launch_bounds__(1024) emit_tiles_sliced(const int32_t* __restr
     off = offsets[e];
     c = offsets[e + 1] - off;
   }
-  emit_tc_tiles(c, off, E, T, has_shared, ts, sh, hdr, (e < E) ? c : ((e == E && has_shared) ? T : 0),
+  emit_tc_tiles(c, E, T, has_shared, ts, sh, hdr, (e < E) ? c : ((e == E && has_shared) ? T : 0),
                 (e < E) ? off : 0, (int)blockIdx.x, (int)gridDim.x);
 }
 
