@@ -14,9 +14,9 @@
 // library holds its kNoAllocScratchBytes until the process exits. Host code
 // cannot use the variable's name as a device address, so the first call on
 // each device resolves the address with cudaGetSymbolAddress (with that
-// device current) and caches it; make that first call before any stream
-// capture. All calls share the one array, so calls that overlap on the GPU
-// (other streams, other host threads) race and corrupt each other's scratch.
+// device current) and caches it. All calls share the one array, so calls
+// that overlap on the GPU (other streams, other host threads) race and
+// corrupt each other's scratch.
 // Every scratch word a call reads is written earlier in the same call, so
 // nothing has to be cleared between calls.
 #include <mutex>

@@ -184,9 +184,9 @@ moe_status moe_dispatch(const moe_layer_desc* desc, const int32_t* topk_idx, int
  * process exits. Limit: T*K <= 65536 (plus the usual E <= 512, K <= 16);
  * larger batches return MOE_ERR_UNSUPPORTED without launching. The first
  * call on a device looks up the array's device address (once per device,
- * with that device current) and caches it: make that first call before any
- * stream capture, and do not call it after cudaDeviceReset on that device
- * (the cached address belongs to the destroyed context). All calls share
+ * with that device current) and caches it: do not call it after
+ * cudaDeviceReset on that device (the cached address belongs to the
+ * destroyed context). All calls share
  * the array, so calls that overlap on the GPU race.
  * Out-of-range indices are handled as in moe_dispatch (inv = -1, perm = -1
  * past the placed copies, counts summing to less than T*K) but are not
